@@ -1,0 +1,242 @@
+"""CPU oracle for tile-routed FP16/INT8 causal prefill attention.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import
+this package.  The product path (``prefill_blockwise_int8_b200``) never
+imports it and shares no code with it.
+
+The arithmetic lives in ``tilemix_oracle.c`` (plain C, fp64, exact integer
+dots); this module compiles it with gcc and marshals numpy arrays.  Each C
+function cites the passage of the TileMix pages it restates.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(closed forms, dense textbook attention in fp64, library attention, brute
+force on tiny inputs, hand-worked quantiser examples in ``tests/golden``).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+_DIR = Path(__file__).resolve().parent
+_SRC = _DIR / "tilemix_oracle.c"
+_LIB_PATH = _DIR / "libtilemix_oracle.so"
+_lib = None
+
+
+def build(force: bool = False) -> Path:
+    """Compile the oracle with gcc (no fast-math, no FMA contraction)."""
+    if force or not _LIB_PATH.exists() or \
+            _LIB_PATH.stat().st_mtime < _SRC.stat().st_mtime:
+        tmp = _LIB_PATH.with_suffix(f".{os.getpid()}.tmp")
+        subprocess.check_call([
+            "gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+            "-ffp-contract=off", "-fno-fast-math", "-D_GNU_SOURCE",
+            str(_SRC), "-o", str(tmp), "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+class _AttnArgs(C.Structure):
+    _fields_ = [
+        ("batch", C.c_int), ("max_seqlen", C.c_int), ("hq", C.c_int),
+        ("hkv", C.c_int), ("d", C.c_int),
+        ("cu_seqlens", C.c_void_p), ("head_map", C.c_void_p),
+        ("q", C.c_void_p), ("q8", C.c_void_p), ("q_scale", C.c_void_p),
+        ("kv_int8", C.c_int),
+        ("k", C.c_void_p), ("k8", C.c_void_p), ("k_scale", C.c_void_p),
+        ("v", C.c_void_p), ("v8", C.c_void_p), ("v_scale", C.c_void_p),
+        ("mask", C.c_void_p), ("block_m", C.c_int), ("block_n", C.c_int),
+        ("group", C.c_int), ("fp16_only", C.c_int),
+        ("quant_block_q", C.c_int), ("quant_block_k", C.c_int),
+        ("softmax_scale", C.c_double),
+        ("out", C.c_void_p), ("lse", C.c_void_p),
+        ("rows", C.c_void_p), ("n_rows", C.c_int64),
+        ("nthreads", C.c_int), ("pair_counts", C.c_void_p),
+    ]
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = C.CDLL(str(build()))
+        lib.oracle_quantize_blockwise.restype = C.c_int
+        lib.oracle_quantize_blockwise.argtypes = [
+            C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int,
+            C.c_int, C.c_void_p, C.c_void_p]
+        lib.oracle_pack_mask.restype = C.c_int
+        lib.oracle_pack_mask.argtypes = [
+            C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int,
+            C.c_int, C.c_int, C.c_void_p]
+        lib.oracle_attn.restype = C.c_int
+        lib.oracle_attn.argtypes = [C.POINTER(_AttnArgs)]
+        lib.oracle_qk_dump.restype = C.c_int
+        lib.oracle_qk_dump.argtypes = [C.POINTER(_AttnArgs), C.c_void_p]
+        lib.oracle_half_to_double.restype = C.c_double
+        lib.oracle_half_to_double.argtypes = [C.c_uint16]
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _c(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def half_to_double(bits: int) -> float:
+    return _load().oracle_half_to_double(bits)
+
+
+def quantize_blockwise(x: np.ndarray, cu_seqlens: np.ndarray, max_seqlen: int,
+                       block: int = 128):
+    """x: float16 [T, H, d] -> (int8 [T, H, d], float32 [H, B, nblk])."""
+    x = _c(x, np.float16)
+    cu = _c(cu_seqlens, np.int32)
+    t, heads, d = x.shape
+    batch = len(cu) - 1
+    nblk = -(-max_seqlen // block)
+    x8 = np.zeros((t, heads, d), dtype=np.int8)
+    scale = np.zeros((heads, batch, nblk), dtype=np.float32)
+    rc = _load().oracle_quantize_blockwise(
+        _ptr(x), _ptr(cu), batch, max_seqlen, heads, d, block, _ptr(x8),
+        _ptr(scale))
+    if rc:
+        raise OracleError(f"oracle_quantize_blockwise failed ({rc})")
+    return x8, scale
+
+
+def pack_mask(route: np.ndarray, cu_seqlens: np.ndarray, max_seqlen: int,
+              block_m: int, block_n: int, group: int) -> np.ndarray:
+    """route: uint8 [B, Hkv, Tm_max, 64] -> uint64 [B, Hkv, Tm_max]."""
+    route = _c(route, np.uint8)
+    cu = _c(cu_seqlens, np.int32)
+    batch, hkv, tm, ng = route.shape
+    if ng != 64 or tm != -(-max_seqlen // block_m):
+        raise OracleError("route must be [batch, hkv, ceil(max_seqlen/BM), 64]")
+    mask = np.zeros((batch, hkv, tm), dtype=np.uint64)
+    rc = _load().oracle_pack_mask(_ptr(route), _ptr(cu), batch, max_seqlen,
+                                  hkv, block_m, block_n, group, _ptr(mask))
+    if rc:
+        raise OracleError(f"oracle_pack_mask failed ({rc})")
+    return mask
+
+
+def _args(cu_seqlens, max_seqlen, q, k=None, v=None, *, q8=None, q_scale=None,
+          k8=None, k_scale=None, v8=None, v_scale=None, mask=None,
+          block_m=128, block_n=128, group=1, head_map=None, fp16_only=False,
+          quant_block_q=128, quant_block_k=128, softmax_scale=None,
+          kv_int8=False, hkv=None):
+    keep = []
+
+    def hold(a, dt):
+        a = _c(a, dt)
+        keep.append(a)
+        return a
+
+    cu = hold(cu_seqlens, np.int32)
+    q = hold(q, np.float16)
+    t, hq, d = q.shape
+    if hkv is None:
+        hkv = (k8 if kv_int8 else k).shape[1]
+    a = _AttnArgs()
+    a.batch, a.max_seqlen, a.hq, a.hkv, a.d = len(cu) - 1, max_seqlen, hq, hkv, d
+    a.cu_seqlens = _ptr(cu)
+    a.head_map = _ptr(hold(head_map, np.int32)) if head_map is not None else None
+    a.q = _ptr(q)
+    a.q8 = _ptr(hold(q8, np.int8)) if q8 is not None else None
+    a.q_scale = _ptr(hold(q_scale, np.float32)) if q_scale is not None else None
+    a.kv_int8 = int(kv_int8)
+    a.k = _ptr(hold(k, np.float16)) if k is not None else None
+    a.k8 = _ptr(hold(k8, np.int8)) if k8 is not None else None
+    a.k_scale = _ptr(hold(k_scale, np.float32)) if k_scale is not None else None
+    a.v = _ptr(hold(v, np.float16)) if v is not None else None
+    a.v8 = _ptr(hold(v8, np.int8)) if v8 is not None else None
+    a.v_scale = _ptr(hold(v_scale, np.float32)) if v_scale is not None else None
+    a.mask = _ptr(hold(mask, np.uint64)) if mask is not None else None
+    a.block_m, a.block_n, a.group = block_m, block_n, group
+    a.fp16_only = int(fp16_only)
+    a.quant_block_q, a.quant_block_k = quant_block_q, quant_block_k
+    a.softmax_scale = (1.0 / np.sqrt(d)) if not softmax_scale else softmax_scale
+    return a, keep, (t, hq, d)
+
+
+def attn_prefill(cu_seqlens, max_seqlen, q, k=None, v=None, *, rows=None,
+                 nthreads=0, want_lse=False, want_pair_counts=False, **kw):
+    """Causal tile-routed attention in fp64.
+
+    Returns out float64 [T, hq, d] (rows not listed in `rows` stay 0), and
+    optionally lse float64 [hq, T] and pair counts (fp16, int8)."""
+    a, keep, (t, hq, d) = _args(cu_seqlens, max_seqlen, q, k, v, **kw)
+    out = np.zeros((t, hq, d), dtype=np.float64)
+    lse = np.zeros((hq, t), dtype=np.float64) if want_lse else None
+    counts = np.zeros(2, dtype=np.int64) if want_pair_counts else None
+    a.out, a.lse = _ptr(out), _ptr(lse)
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        keep.append(rows)
+        a.rows, a.n_rows = _ptr(rows), len(rows)
+    a.nthreads = nthreads
+    a.pair_counts = _ptr(counts)
+    rc = _load().oracle_attn(C.byref(a))
+    if rc:
+        raise OracleError(f"oracle_attn failed ({rc})")
+    res = [out]
+    if want_lse:
+        res.append(lse)
+    if want_pair_counts:
+        res.append(counts)
+    return res[0] if len(res) == 1 else tuple(res)
+
+
+def qk_dump(cu_seqlens, max_seqlen, q8, k8, mask, *, hq, hkv, d, block_m,
+            block_n, group, head_map=None, fill=0):
+    """INT32 accumulators of every INT8-routed legal tile,
+    int32 [B, hq, Tm_max, Tn_max, BM, BN]; untouched entries hold `fill`."""
+    t = q8.shape[0]
+    dummy_q = np.zeros((t, hq, d), dtype=np.float16)
+    a, keep, _ = _args(cu_seqlens, max_seqlen, dummy_q, None, None, q8=q8,
+                       k8=k8, k_scale=np.ones(1, np.float32),
+                       q_scale=np.ones(1, np.float32), mask=mask,
+                       block_m=block_m, block_n=block_n, group=group,
+                       head_map=head_map, hkv=hkv)
+    tm = -(-max_seqlen // block_m)
+    tn = -(-max_seqlen // block_n)
+    dump = np.full((len(cu_seqlens) - 1, hq, tm, tn, block_m, block_n), fill,
+                   dtype=np.int32)
+    rc = _load().oracle_qk_dump(C.byref(a), _ptr(dump))
+    if rc:
+        raise OracleError(f"oracle_qk_dump failed ({rc})")
+    return dump
+
+
+def prepare(inputs: dict, fp16_only: bool = False):
+    """Run the oracle's own quantiser and packer on generator output and
+    return the keyword arguments of `attn_prefill` for that workload."""
+    w = inputs["workload"]
+    cu, ms = inputs["cu_seqlens"], inputs["max_seqlen"]
+    q8, sq = quantize_blockwise(inputs["q"], cu, ms, w.quant_block_q)
+    k8, sk = quantize_blockwise(inputs["k"], cu, ms, w.quant_block_k)
+    mask = pack_mask(inputs["route"], cu, ms, w.block_m, w.block_n,
+                     inputs["group"])
+    kw = dict(q8=q8, q_scale=sq, k8=k8, k_scale=sk, mask=mask,
+              block_m=w.block_m, block_n=w.block_n, group=inputs["group"],
+              quant_block_q=w.quant_block_q, quant_block_k=w.quant_block_k,
+              fp16_only=fp16_only)
+    if w.kv_format == "int8":
+        v8, sv = quantize_blockwise(inputs["v"], cu, ms, w.quant_block_k)
+        kw.update(kv_int8=True, v8=v8, v_scale=sv)
+        args = (cu, ms, inputs["q"], None, None)
+    else:
+        args = (cu, ms, inputs["q"], inputs["k"], inputs["v"])
+    return args, kw

@@ -1,0 +1,407 @@
+"""Pins for the CPU oracle: each test ties it to something other than itself.
+
+* binary16 decoding against numpy's IEEE conversion (all 65536 patterns);
+* the quantiser against hand-worked examples (tests/golden) and the
+  invariants of blockwise symmetric rounding;
+* the packer against the shift-and-mask lookup R = (b >> g_j) & 1 of the
+  gist.science technical summary on hand-built words, and brute force;
+* attention against dense fp64 textbook attention softmax(QK^T/sqrt(d))V
+  with a causal mask (section 3 Preliminaries), against torch's
+  scaled_dot_product_attention in float64, against brute-force attention on
+  dequantised operands, against an explicit materialise-then-softmax score
+  matrix with the routing expanded tile by tile, and against closed forms
+  (rows of P sum to 1, row 0 returns v_0, linearity in V).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------
+# independent dense references (no oracle code)
+# ----------------------------------------------------------------------------
+
+def dense_attention(q, k, v, scale, scores=None):
+    """Textbook causal attention of one sequence in fp64.
+    q [L, Hq, d], k/v [L, Hkv, d] (contiguous GQA groups)."""
+    L, hq, d = q.shape
+    hkv = k.shape[1]
+    rep = hq // hkv
+    out = np.zeros((L, hq, d))
+    lse = np.zeros((hq, L))
+    causal = np.tril(np.ones((L, L), dtype=bool))
+    for h in range(hq):
+        qh = q[:, h, :].astype(np.float64)
+        kh = k[:, h // rep, :].astype(np.float64)
+        vh = v[:, h // rep, :].astype(np.float64)
+        s = scale * (qh @ kh.T) if scores is None else scores(h)
+        s = np.where(causal, s, -np.inf)
+        mu = s.max(axis=1, keepdims=True)
+        p = np.exp(s - mu)
+        out[:, h, :] = (p @ vh) / p.sum(axis=1, keepdims=True)
+        lse[h] = mu[:, 0] + np.log(p.sum(axis=1))
+    return out, lse
+
+
+def expand_scales(scale, heads_first_index, length, block):
+    """Per-token scale of one head/sequence from [nblk] block scales."""
+    return np.repeat(scale, block)[:length].astype(np.float64)
+
+
+def tiny_inputs(L=256, hq=2, hkv=1, d=64, seed=11, outliers=False):
+    w = W.TINY.with_(seqlen=L, hq=hq, hkv=hkv, d=d, seed=seed,
+                     outliers=outliers)
+    return W.make(w)
+
+
+# ----------------------------------------------------------------------------
+# binary16
+# ----------------------------------------------------------------------------
+
+def test_half_decoding_all_patterns():
+    bits = np.arange(1 << 16, dtype=np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([oracle.half_to_double(int(b)) for b in bits])
+    finite = np.isfinite(ref)
+    assert np.array_equal(got[finite], ref[finite])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.array_equal(got[np.isinf(ref)], ref[np.isinf(ref)])
+
+
+# ----------------------------------------------------------------------------
+# quantiser
+# ----------------------------------------------------------------------------
+
+def test_quantiser_golden_examples():
+    with open(os.path.join(GOLDEN, "quantize_examples.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        x = np.array(c["x"], dtype=np.float16)          # [tokens, d]
+        L, d = x.shape
+        x3 = x.reshape(L, 1, d)
+        cu = np.array([0, L], dtype=np.int32)
+        q8, s = oracle.quantize_blockwise(x3, cu, L, block=L)
+        assert s.shape == (1, 1, 1)
+        assert s[0, 0, 0] == np.float32(c["scale"]), c["name"]
+        if "scale_hex" in c:
+            assert float(s[0, 0, 0]).hex() == c["scale_hex"]
+        assert np.array_equal(q8.reshape(L, d), np.array(c["q"])), c["name"]
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_quantiser_invariants_varlen(block):
+    lens = np.array([1, 127, 128, 129, 300], dtype=np.int32)
+    cu = W.cu_seqlens(lens)
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((lens.sum(), 3, 64)) * 3).astype(np.float16)
+    x[cu[2]:cu[3], 1, :] = 0  # one all-zero block
+    q8, s = oracle.quantize_blockwise(x, cu, int(lens.max()), block=block)
+    nblk = -(-int(lens.max()) // block)
+    assert s.shape == (3, len(lens), nblk)
+    for b in range(len(lens)):
+        for h in range(3):
+            for t in range(nblk):
+                r0, r1 = t * block, min((t + 1) * block, int(lens[b]))
+                if r0 >= lens[b]:
+                    assert s[h, b, t] == 0
+                    continue
+                blk = x[cu[b] + r0:cu[b] + r1, h, :].astype(np.float32)
+                qb = q8[cu[b] + r0:cu[b] + r1, h, :].astype(np.int32)
+                a = np.abs(blk).max()
+                if a == 0:
+                    assert s[h, b, t] == 0 and not qb.any()
+                    continue
+                sc = np.float64(s[h, b, t])
+                # scale is absmax/127 to fp32 accuracy
+                assert abs(sc * 127 - a) <= a * 2.0 ** -23
+                # the absmax element maps to +-127, codes stay in range
+                assert np.abs(qb).max() == 127
+                assert np.abs(qb).max() <= 127
+                # every code is a nearest integer of x / scale, up to the
+                # fp32 rounding of the quotient (|x/s| <= 127, half an ulp)
+                err = np.abs(blk.astype(np.float64) - qb * sc)
+                assert (err <= sc * (0.5 + 128 * 2.0 ** -24)).all()
+
+
+# ----------------------------------------------------------------------------
+# packer
+# ----------------------------------------------------------------------------
+
+def test_pack_shift_and_mask_lookup_hand_built():
+    # one sequence of 300 tokens, BM=64, BN=32, g=2: Tm=5
+    L, bm, bn, g = 300, 64, 32, 2
+    cu = np.array([0, L], dtype=np.int32)
+    tm = -(-L // bm)
+    route = np.zeros((1, 1, tm, 64), dtype=np.uint8)
+    pattern = [1, 0, 1, 1, 0, 1, 0, 0, 1, 1]
+    for m in range(tm):
+        route[0, 0, m, :len(pattern)] = pattern
+    route[0, 0, :, 40] = 7   # far beyond any legal group: must be cleared
+    mask = oracle.pack_mask(route, cu, L, bm, bn, g)
+    for m in range(tm):
+        word = int(mask[0, 0, m])
+        last_row = min((m + 1) * bm, L) - 1
+        n_last = last_row // bn
+        for n in range(n_last + 1):
+            # R_{hk,m,g_j} = (b_{hk,m} >> g_j) & 1 with g_j = floor(n / g)
+            assert (word >> (n // g)) & 1 == (route[0, 0, m, n // g] != 0)
+        assert word >> (n_last // g + 1) == 0  # illegal groups carry 0
+    # m = 0: rows 0..63, keys 0..63 -> tiles 0,1 -> group 0 only
+    assert int(mask[0, 0, 0]) == 0b1
+    # m = 4: rows 256..299 -> tiles 0..9 -> groups 0..4 -> bits 1,0,1,1,0
+    assert int(mask[0, 0, 4]) == 0b01101
+
+
+def test_pack_bruteforce_all_workload_shapes():
+    for w in [W.TINY, W.LLAMA32_3B_4K, W.VARLEN16, W.INT8KV_16K,
+              W.sweep_32k(50)]:
+        lens = W.seqlens(w)
+        cu = W.cu_seqlens(lens)
+        g = W.group_size(w, lens)
+        route = W.route_bytes(w, lens, junk_in_illegal=True)
+        clean = W.route_bytes(w, lens)
+        mask = oracle.pack_mask(route, cu, int(lens.max()), w.block_m,
+                                w.block_n, g)
+        bits = ((mask[..., None] >> np.arange(64, dtype=np.uint64)) & 1)
+        assert np.array_equal(bits.astype(np.uint8), clean)
+        assert int(bits.sum()) == int(clean.sum())
+
+
+def test_pack_rejects_more_than_64_groups():
+    L = 64 * 65
+    cu = np.array([0, L], dtype=np.int32)
+    route = np.zeros((1, 1, L // 64, 64), dtype=np.uint8)
+    with pytest.raises(oracle.OracleError):
+        oracle.pack_mask(route, cu, L, 64, 64, 1)
+
+
+# ----------------------------------------------------------------------------
+# attention
+# ----------------------------------------------------------------------------
+
+def run(inp, **kw):
+    args, okw = oracle.prepare(inp, fp16_only=kw.pop("fp16_only", False))
+    okw.update(kw)
+    return oracle.attn_prefill(*args, **okw), okw
+
+
+@pytest.mark.parametrize("hq,hkv,d", [(2, 1, 64), (4, 2, 32), (3, 3, 16)])
+def test_all_fp16_equals_dense_textbook(hq, hkv, d):
+    inp = tiny_inputs(L=160, hq=hq, hkv=hkv, d=d)
+    (out, lse), _ = run(inp, fp16_only=True, want_lse=True)
+    ref, ref_lse = dense_attention(inp["q"], inp["k"], inp["v"],
+                                   1.0 / np.sqrt(d))
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+def test_all_zero_mask_equals_fp16_only():
+    inp = tiny_inputs()
+    inp["route"][:] = 0
+    a, _ = run(inp)
+    b, _ = run(inp, fp16_only=True)
+    assert np.array_equal(a, b)
+
+
+def test_all_fp16_equals_torch_sdpa_float64():
+    torch = pytest.importorskip("torch")
+    inp = tiny_inputs(L=200, hq=4, hkv=2, d=32)
+    out, _ = run(inp, fp16_only=True)
+    q = torch.from_numpy(inp["q"].astype(np.float64)).permute(1, 0, 2)
+    k = torch.from_numpy(inp["k"].astype(np.float64)).permute(1, 0, 2)
+    v = torch.from_numpy(inp["v"].astype(np.float64)).permute(1, 0, 2)
+    k = k.repeat_interleave(2, dim=0)
+    v = v.repeat_interleave(2, dim=0)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q[None], k[None], v[None], is_causal=True)[0].permute(1, 0, 2)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("qb,kb", [(128, 128), (128, 64), (64, 32)])
+def test_all_int8_equals_dequantised_dense(qb, kb):
+    inp = tiny_inputs(L=256, hq=4, hkv=2, d=64, outliers=True)
+    inp["workload"] = inp["workload"].with_(quant_block_q=qb, quant_block_k=kb)
+    inp["route"][:] = 1
+    out, okw = run(inp)
+    L, d = 256, 64
+    qhat = np.zeros((L, 4, d))
+    khat = np.zeros((L, 2, d))
+    for h in range(4):
+        qhat[:, h] = okw["q8"][:, h].astype(np.float64) * \
+            expand_scales(okw["q_scale"][h, 0], h, L, qb)[:, None]
+    for h in range(2):
+        khat[:, h] = okw["k8"][:, h].astype(np.float64) * \
+            expand_scales(okw["k_scale"][h, 0], h, L, kb)[:, None]
+    ref, _ = dense_attention(qhat, khat, inp["v"], 1.0 / np.sqrt(d))
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("bm,bn,g", [(64, 64, 1), (128, 64, 1), (64, 32, 2),
+                                     (128, 128, 1), (32, 64, 3)])
+def test_mixed_mask_equals_materialised_scores(bm, bn, g):
+    L, hq, hkv, d = 256, 2, 1, 64
+    inp = tiny_inputs(L=L, hq=hq, hkv=hkv, d=d, outliers=True)
+    w = inp["workload"].with_(block_m=bm, block_n=bn, group=g)
+    inp["workload"], inp["group"] = w, g
+    inp["route"] = W.route_bytes(w, inp["seqlens"])
+    out, okw = run(inp)
+    scale = 1.0 / np.sqrt(d)
+    q, k = inp["q"].astype(np.float64), inp["k"].astype(np.float64)
+    sq = expand_scales(okw["q_scale"][0, 0], 0, L, 128)
+    sk = expand_scales(okw["k_scale"][0, 0], 0, L, 128)
+    tm, tn = -(-L // bm), -(-L // bn)
+    # route of every (query tile, key tile), expanded to elements
+    tile_route = np.zeros((tm, tn))
+    for m in range(tm):
+        for n in range(tn):
+            tile_route[m, n] = inp["route"][0, 0, m, n // g] if n // g < 64 else 0
+    R = np.kron(tile_route, np.ones((bm, bn)))[:L, :L].astype(bool)
+
+    def scores(h):
+        s16 = scale * (q[:, h] @ k[:, 0].T)
+        s8 = scale * (okw["q8"][:, h].astype(np.float64) @
+                      okw["k8"][:, 0].astype(np.float64).T) * \
+            np.outer(sq if h == 0 else expand_scales(okw["q_scale"][h, 0], h, L, 128), sk)
+        return np.where(R, s8, s16)
+
+    ref, _ = dense_attention(inp["q"], inp["k"], inp["v"], scale, scores)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-11)
+    # the route really mixes both paths here
+    assert 0 < R[np.tril_indices(L)].mean() < 1
+
+
+def test_probability_rows_sum_to_one_and_row0_is_v0():
+    inp = tiny_inputs(outliers=True)
+    inp["v"] = np.ones_like(inp["v"])
+    out, _ = run(inp)
+    np.testing.assert_allclose(out, 1.0, rtol=0, atol=1e-12)
+    inp2 = tiny_inputs(outliers=True)
+    out2, _ = run(inp2)
+    assert np.array_equal(out2[0, 0], inp2["v"][0, 0].astype(np.float64))
+    assert np.array_equal(out2[0, 1], inp2["v"][0, 0].astype(np.float64))
+
+
+def test_linear_in_v():
+    inp = tiny_inputs(outliers=True)
+    out, _ = run(inp)
+    inp["v"] = (inp["v"].astype(np.float32) * 2).astype(np.float16)
+    out2, _ = run(inp)
+    np.testing.assert_allclose(out2, 2 * out, rtol=1e-13, atol=0)
+
+
+def test_group_two_equals_duplicated_bits_group_one():
+    L, bm, bn = 256, 64, 32
+    inp = tiny_inputs(L=L)
+    w2 = inp["workload"].with_(block_m=bm, block_n=bn, group=2)
+    r2 = W.route_bytes(w2, inp["seqlens"])
+    r1 = np.zeros_like(r2)
+    r1[..., 0::2] = r2[..., :32]
+    r1[..., 1::2] = r2[..., :32]
+    inp["workload"], inp["group"], inp["route"] = w2, 2, r2
+    a, _ = run(inp)
+    inp["workload"], inp["group"], inp["route"] = w2.with_(group=1), 1, r1
+    b, _ = run(inp)
+    assert np.array_equal(a, b)
+
+
+def test_varlen_sequences_are_independent():
+    w = W.VARLEN16.with_(batch=3, varlen_lo=1, varlen_hi=200, hq=4, hkv=2,
+                         d=32, block_m=64, block_n=32, group=0)
+    inp = W.make(w)
+    out, _ = run(inp)
+    lens, cu = inp["seqlens"], inp["cu_seqlens"]
+    for b in range(3):
+        sub = dict(inp)
+        sl = slice(cu[b], cu[b + 1])
+        sub.update(seqlens=lens[b:b + 1], cu_seqlens=np.array([0, lens[b]], np.int32),
+                   max_seqlen=int(lens.max()), q=inp["q"][sl], k=inp["k"][sl],
+                   v=inp["v"][sl], route=inp["route"][b:b + 1])
+        sub["workload"] = w.with_(batch=1)
+        o_b, _ = run(sub)
+        assert np.array_equal(o_b, out[sl])
+
+
+def test_explicit_head_map_equals_contiguous():
+    inp = tiny_inputs(L=128, hq=6, hkv=2, d=32, outliers=True)
+    a, _ = run(inp)
+    b, _ = run(inp, head_map=np.array([0, 0, 0, 1, 1, 1], np.int32))
+    assert np.array_equal(a, b)
+    c, _ = run(inp, head_map=np.array([1, 1, 1, 0, 0, 0], np.int32))
+    assert not np.array_equal(a, c)
+
+
+def test_int8_kv_cache_equals_dequantised_dense():
+    inp = tiny_inputs(L=256, hq=2, hkv=2, d=64, outliers=True)
+    w = inp["workload"].with_(kv_format="int8", block_m=128, block_n=128,
+                              group=1)
+    inp["workload"] = w
+    inp["route"] = W.route_bytes(w, inp["seqlens"])
+    out, okw = run(inp)
+    L, d, scale = 256, 64, 1 / 8.0
+    khat = np.zeros((L, 2, d))
+    vhat = np.zeros((L, 2, d))
+    for h in range(2):
+        ks = expand_scales(okw["k_scale"][h, 0], h, L, 128)[:, None]
+        vs = expand_scales(okw["v_scale"][h, 0], h, L, 128)[:, None]
+        khat[:, h] = okw["k8"][:, h] * ks
+        vhat[:, h] = okw["v8"][:, h] * vs
+    def scores(h):  # MHA: query head h reads KV head h and its routing
+        R = np.kron(inp["route"][0, h, :2, :2].astype(float),
+                    np.ones((128, 128))).astype(bool)
+        s16 = scale * (inp["q"][:, h].astype(np.float64) @ khat[:, h].T)
+        sq = expand_scales(okw["q_scale"][h, 0], h, L, 128)
+        s8 = scale * (okw["q8"][:, h].astype(np.float64) @ khat[:, h].T) * sq[:, None]
+        return np.where(R, s8, s16)
+
+    ref, _ = dense_attention(inp["q"], khat, vhat, scale, scores)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-11)
+
+
+def test_row_sample_matches_full_run():
+    inp = tiny_inputs(outliers=True)
+    full, _ = run(inp)
+    rows = np.array([0, 1, 63, 64, 200, 255])
+    part, _ = run(inp, rows=rows)
+    assert np.array_equal(part[rows], full[rows])
+    others = np.setdiff1d(np.arange(256), rows)
+    assert not part[others].any()
+
+
+def test_pair_counts():
+    inp = tiny_inputs()
+    inp["route"][:] = 1
+    (_, counts), _ = run(inp, want_pair_counts=True)
+    assert counts[0] == 0 and counts[1] == 2 * 256 * 257 // 2
+    inp["route"][:] = 0
+    (_, counts), _ = run(inp, want_pair_counts=True)
+    assert counts[1] == 0 and counts[0] == 2 * 256 * 257 // 2
+
+
+def test_qk_dump_equals_integer_matmul():
+    inp = tiny_inputs(outliers=True)
+    args, okw = oracle.prepare(inp)
+    w = inp["workload"]
+    dump = oracle.qk_dump(inp["cu_seqlens"], 256, okw["q8"], okw["k8"],
+                          okw["mask"], hq=2, hkv=1, d=64, block_m=64,
+                          block_n=64, group=1, fill=-1)
+    full = [okw["q8"][:, h].astype(np.int64) @ okw["k8"][:, 0].astype(np.int64).T
+            for h in range(2)]
+    seen = 0
+    for h in range(2):
+        for m in range(4):
+            for n in range(4):
+                tile = dump[0, h, m, n]
+                routed = inp["route"][0, 0, m, n] and n <= m
+                if routed:
+                    assert np.array_equal(tile, full[h][m*64:(m+1)*64, n*64:(n+1)*64])
+                    seen += 1
+                else:
+                    assert (tile == -1).all()
+    assert seen > 0
