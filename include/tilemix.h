@@ -1,0 +1,217 @@
+/*
+ * tilemix.h - C ABI of the tile-routed FP16/INT8 causal prefill attention
+ * library for NVIDIA B200 (sm_100a).
+ *
+ * The operation follows "TileMix: Tile-Centric Mixed-Precision Attention for
+ * LLM Inference Acceleration" (arXiv 2608.17336) as summarised on its public
+ * pages.  The causal score matrix of every sequence is cut into BM x BN score
+ * tiles; one 64-bit routing word per (sequence, KV head, query-tile row)
+ * carries one bit per group of g adjacent key tiles; a legal tile group whose
+ * bit is 1 computes its scores as Q8 K8^T on INT8 tensor cores with INT32
+ * accumulation, rescaled by the two block scales, and one whose bit is 0
+ * computes them as Q K^T in FP16; both feed the same online-softmax state and
+ * the FP16 P V product.
+ *
+ * Conventions shared by every call:
+ *  - Pointers marked "dev" are CUDA device pointers, owned by the caller,
+ *    which must keep them alive until the stream work completes.  The
+ *    library allocates nothing, never synchronises the device or the stream,
+ *    and copies nothing between host and device.
+ *  - Every call is asynchronous on `stream` (NULL = the legacy default
+ *    stream) and returns after enqueueing its kernels.
+ *  - Token-major, unpadded layout: a tensor "[T, H, d]" holds the T = sum of
+ *    all sequence lengths tokens back to back, each token's H heads back to
+ *    back, each head's d channels contiguous.  Sequence b spans tokens
+ *    [cu_seqlens[b], cu_seqlens[b+1]).
+ *  - Argument errors are detected on the host before anything is launched;
+ *    the call then returns a status other than TILEMIX_OK, launches nothing,
+ *    and tilemix_last_error() describes the problem.
+ *  - Problems only the device can see (a non-monotone cu_seqlens, a length
+ *    above max_seqlen, a head_map entry out of range, a pipeline wait that
+ *    ran past its time limit) are reported through the optional `status`
+ *    word (dev int32): the first kernel to see one stores its
+ *    tilemix_status code there (if the word is still 0) and its blocks
+ *    return without touching the outputs they would have written; blocks
+ *    of tilemix_attn_prefill that start while the word is nonzero return at
+ *    once.  The caller zeroes the word before the call and reads it after
+ *    the stream work completes.  Kernels never trap.
+ *  - Inputs must be finite.  NaN or Inf input gives undefined output.
+ */
+#ifndef TILEMIX_H_
+#define TILEMIX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* tilemix_stream_t;
+
+typedef enum {
+  TILEMIX_OK = 0,
+  TILEMIX_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size       */
+  TILEMIX_ERR_UNSUPPORTED = 2,  /* valid but not built (d, tile shape ...) */
+  TILEMIX_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed       */
+  TILEMIX_ERR_TIMEOUT = 4,      /* device: a pipeline wait ran too long    */
+  TILEMIX_ERR_BAD_SEQLENS = 5,  /* device: cu_seqlens or head_map invalid  */
+  TILEMIX_ERR_NO_DEVICE = 6     /* current device is not sm_100            */
+} tilemix_status;
+
+enum { TILEMIX_KV_FP16 = 0, TILEMIX_KV_INT8 = 1 };
+
+/* Ignore the routing words: every legal tile takes the FP16 path and the
+ * INT8 operands (q8, q_scale, and k8, k_scale for TILEMIX_KV_FP16) may be
+ * NULL.  This is the all-FP16 reference mode. */
+#define TILEMIX_FLAG_FP16_ONLY 1u
+
+/*
+ * Blockwise symmetric INT8 quantisation ("quantize-once").
+ * Pages: section 3 Preliminaries (blockwise quantization; INT8 tensor cores
+ * with INT32 accumulation) and appendix C Quantization Configuration
+ * (blockwise symmetric INT8 of Q and K, made once per attention call).
+ *
+ * For every sequence b, head h and block t of `block` consecutive tokens of
+ * that sequence (blocks restart at each sequence start; the last block of a
+ * sequence may be short):
+ *   a = max |x| over the block's tokens and d channels,
+ *   scale[h][b][t] = a / 127            (one IEEE fp32 division),
+ *   x8 = clamp(round_half_even(x / scale), -127, 127) (IEEE fp32 division),
+ *   a == 0 gives scale 0 and codes 0.
+ * Blocks t >= ceil(len_b / block) of a shorter sequence get scale 0.
+ *
+ *   x          dev fp16 [T, heads, head_dim], 16-byte aligned
+ *   cu_seqlens dev int32 [batch + 1], non-decreasing, cu_seqlens[0] = 0
+ *   max_seqlen host int: >= every sequence length
+ *   total_tokens host int: T = cu_seqlens[batch], the rows of x and x8
+ *   head_dim   multiple of 8, <= 256; block in [1, 256], block*head_dim <= 32768
+ *   x8         dev int8 [T, heads, head_dim], 16-byte aligned
+ *   scale      dev fp32 [heads, batch, ceil(max_seqlen / block)]
+ *   status     optional dev int32 (see above)
+ */
+tilemix_status tilemix_quantize_blockwise(
+    const void* x, const int32_t* cu_seqlens, int batch, int max_seqlen,
+    int total_tokens, int heads, int head_dim, int block, int8_t* x8,
+    float* scale, int32_t* status, tilemix_stream_t stream);
+
+/*
+ * Pack per-group routing bytes into 64-bit routing words.
+ * Pages: section 3 Preliminaries (packed 64-bit masks, bit floor(n/g) of the
+ * word of a query-tile row selects the path of key tile n), section 4
+ * (routing map indexed by KV head, query-tile row and key-tile group), and
+ * the gist.science technical summary (lookup R = (b >> g_j) & 1).
+ *
+ * Output bit j of word [b][hk][m] is (route[b][hk][m][j] != 0) for every
+ * group j that holds a legal (causal, in-sequence) query/key pair of
+ * query-tile row m; every other bit is 0 (junk in illegal groups is
+ * cleared).  1 = INT8, 0 = FP16.
+ *
+ *   route      dev uint8 [batch, hkv, Tm_max, 64], Tm_max = ceil(max_seqlen/block_m)
+ *   block_m, block_n  score-tile shape the words will be read with
+ *   group      g >= 1 with ceil(ceil(max_seqlen / block_n) / g) <= 64
+ *   mask       dev uint64 [batch, hkv, Tm_max], 8-byte aligned
+ */
+tilemix_status tilemix_pack_mask(
+    const uint8_t* route, const int32_t* cu_seqlens, int batch,
+    int max_seqlen, int hkv, int block_m, int block_n, int group,
+    uint64_t* mask, int32_t* status, tilemix_stream_t stream);
+
+/*
+ * Arguments of tilemix_attn_prefill.  Zero-initialise, set struct_size =
+ * sizeof(tilemix_attn_params), then fill the fields.
+ */
+typedef struct {
+  uint32_t struct_size;
+  int kv_format;        /* TILEMIX_KV_FP16 or TILEMIX_KV_INT8 (INT8 cache)  */
+  uint32_t flags;       /* TILEMIX_FLAG_*                                    */
+
+  /* Q: fp16 [T, hq, d]; Q8: int8 [T, hq, d]; q_scale: fp32
+   * [hq, batch, ceil(max_seqlen / quant_block_q)] (tilemix_quantize_blockwise
+   * output).  All 16-byte aligned. */
+  const void* q;
+  const int8_t* q8;
+  const float* q_scale;
+  /* TILEMIX_KV_FP16: k, v fp16 [T, hkv, d]; k8 + k_scale (as for Q, block
+   * quant_block_k) for INT8-routed groups.
+   * TILEMIX_KV_INT8: k8, v8 int8 [T, hkv, d] with k_scale, v_scale fp32
+   * [hkv, batch, ceil(max_seqlen / quant_block_k)]; k and v unused.  FP16
+   * groups then use K = k8 * k_scale exactly; V = v8 * v_scale always. */
+  const void* k;
+  const int8_t* k8;
+  const float* k_scale;
+  const void* v;
+  const int8_t* v8;
+  const float* v_scale;
+
+  const int32_t* cu_seqlens; /* dev int32 [batch + 1]                      */
+  int batch;
+  int max_seqlen;            /* host: >= every sequence length              */
+  int total_tokens;          /* host: T = cu_seqlens[batch]; the kernels
+                                never address a token row at or past T    */
+  int hq, hkv, head_dim;     /* head_dim in {64, 128}                       */
+  /* dev int32 [hq]: KV head of each query head (query heads mapped to one
+   * KV head share its K, V and routing words).  NULL: contiguous groups,
+   * KV head = h / (hq / hkv), which needs hq % hkv == 0. */
+  const int32_t* head_map;
+
+  /* Routing words from tilemix_pack_mask: dev uint64 [batch, hkv,
+   * ceil(max_seqlen / block_m)].  Tile shape: block_m in {64, 128},
+   * block_n in {64, 128} (block_m = 64 needs block_n = 64), group g >= 1
+   * with ceil(ceil(max_seqlen / block_n) / g) <= 64.  Bits of illegal groups
+   * are ignored. */
+  const uint64_t* mask;
+  int block_m, block_n, group;
+  /* Quantisation block lengths in tokens: quant_block_q >= 1, quant_block_k
+   * a multiple of block_n (one K scale per key tile). 0 = 128. */
+  int quant_block_q, quant_block_k;
+  float softmax_scale;       /* > 0; <= 0 means 1 / sqrt(head_dim)         */
+  int causal;                /* must be 1                                   */
+
+  void* out;                 /* dev fp16 [T, hq, d]                         */
+  float* lse;                /* optional dev fp32 [hq, T]: natural-log LSE  */
+  /* Optional debug output, dev int32 [batch, hq, Tm_max, Tn_max, block_m,
+   * block_n] with Tn_max = ceil(max_seqlen / block_n): the raw INT32
+   * accumulators of every INT8-routed legal tile, written for rows inside
+   * the sequence; entries of other tiles are left untouched. */
+  int32_t* qk_dump;
+  int32_t* status;           /* optional dev int32, see above               */
+} tilemix_attn_params;
+
+/*
+ * Causal tile-routed prefill attention (forward, GQA, unpadded varlen).
+ * Pages: section 3 Preliminaries (S = QK^T, P = softmax(S), O = PV; online
+ * softmax with row maxima and normalisers; FP16 and INT8 score tiles enter a
+ * common domain before updating one maximum, normaliser and accumulator;
+ * routing words and legality), section 4 (GQA and varlen routing),
+ * appendices B-D (legality separate from routing; FP16 V/PV; quantize-once
+ * operands; INT8 KV cache), ainews summary (shared online-softmax state).
+ *
+ * For query i and key j <= i of sequence b, query head h, KV head hk:
+ *   route = bit floor(floor(j / block_n) / group) of
+ *           mask[b][hk][floor(i / block_m)]            (1 = INT8)
+ *   s_ij  = scale * sum_c q8_ic k8_jc * q_scale[h][b][i / qb] * k_scale[hk][b][j / kb]
+ *           if route, else scale * sum_c q_ic k_jc
+ *   out_i = sum_j softmax_j(s_i.) v_j ,  lse_i = ln sum_j exp(s_ij)
+ * computed on sm_100a tensor cores (FP16 MMA with f32 accumulation, INT8
+ * MMA with INT32 accumulation, FP16 P with f32 accumulation for P V).
+ * Returns TILEMIX_ERR_NO_DEVICE when the current device is not sm_100.
+ */
+tilemix_status tilemix_attn_prefill(const tilemix_attn_params* params,
+                                    tilemix_stream_t stream);
+
+/* Static description of a status code. */
+const char* tilemix_status_string(tilemix_status status);
+
+/* Detail of the last error returned on the calling host thread ("" if none). */
+const char* tilemix_last_error(void);
+
+/* Library ABI version: (major << 16) | minor. */
+uint32_t tilemix_version(void);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* TILEMIX_H_ */

@@ -34,7 +34,7 @@ def build(force: bool = False) -> Path:
             _LIB_PATH.stat().st_mtime < _SRC.stat().st_mtime:
         tmp = _LIB_PATH.with_suffix(f".{os.getpid()}.tmp")
         subprocess.check_call([
-            "gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+            "gcc", "-O3", "-std=c11", "-fPIC", "-shared", "-pthread",
             "-ffp-contract=off", "-fno-fast-math", "-D_GNU_SOURCE",
             str(_SRC), "-o", str(tmp), "-lm"])
         os.replace(tmp, _LIB_PATH)

@@ -1,0 +1,259 @@
+"""Tile-routed FP16/INT8 causal prefill attention on B200 (sm_100a).
+
+Thin Python binding of the C ABI in ``include/tilemix.h`` (``libtilemix.so``,
+built in-tree by ``python -m prefill_blockwise_int8_b200.build``).  This
+module only marshals arguments: it takes torch tensors that already live on
+the GPU, passes their device pointers and the current CUDA stream, and
+raises ``TilemixError`` when a call returns a non-OK status.  Every step of
+the computation runs in the library's CUDA kernels; there is no CPU or
+PyTorch fallback, and importing this package fails loudly when the library
+is missing.
+
+Entry points (same names as the C ABI):
+  tilemix_quantize_blockwise(x, cu_seqlens, max_seqlen, block=128)
+      -> (x8, scale)
+  tilemix_pack_mask(route, cu_seqlens, max_seqlen, block_m, block_n, group)
+      -> mask
+  tilemix_attn_prefill(q, k, v, cu_seqlens, max_seqlen, ...) -> out
+"""
+from __future__ import annotations
+
+import ctypes as C
+from pathlib import Path
+
+__all__ = [
+    "TilemixError", "lib", "library_path", "EXPORTED_SYMBOLS",
+    "tilemix_quantize_blockwise", "tilemix_pack_mask", "tilemix_attn_prefill",
+    "tilemix_status_string", "tilemix_last_error", "tilemix_version",
+    "KV_FP16", "KV_INT8", "FLAG_FP16_ONLY", "STATUS",
+]
+
+_LIB_PATH = Path(__file__).resolve().parent / "libtilemix.so"
+
+KV_FP16, KV_INT8 = 0, 1
+FLAG_FP16_ONLY = 1
+STATUS = {0: "TILEMIX_OK", 1: "TILEMIX_ERR_INVALID_ARG",
+          2: "TILEMIX_ERR_UNSUPPORTED", 3: "TILEMIX_ERR_CUDA",
+          4: "TILEMIX_ERR_TIMEOUT", 5: "TILEMIX_ERR_BAD_SEQLENS",
+          6: "TILEMIX_ERR_NO_DEVICE"}
+
+# Every function include/tilemix.h declares.
+EXPORTED_SYMBOLS = (
+    "tilemix_quantize_blockwise", "tilemix_pack_mask", "tilemix_attn_prefill",
+    "tilemix_status_string", "tilemix_last_error", "tilemix_version",
+)
+
+
+class TilemixError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {detail}")
+        self.status = status
+
+
+class AttnParams(C.Structure):
+    """Mirror of tilemix_attn_params (include/tilemix.h)."""
+    _fields_ = [
+        ("struct_size", C.c_uint32), ("kv_format", C.c_int),
+        ("flags", C.c_uint32),
+        ("q", C.c_void_p), ("q8", C.c_void_p), ("q_scale", C.c_void_p),
+        ("k", C.c_void_p), ("k8", C.c_void_p), ("k_scale", C.c_void_p),
+        ("v", C.c_void_p), ("v8", C.c_void_p), ("v_scale", C.c_void_p),
+        ("cu_seqlens", C.c_void_p), ("batch", C.c_int),
+        ("max_seqlen", C.c_int), ("total_tokens", C.c_int),
+        ("hq", C.c_int), ("hkv", C.c_int), ("head_dim", C.c_int),
+        ("head_map", C.c_void_p),
+        ("mask", C.c_void_p), ("block_m", C.c_int), ("block_n", C.c_int),
+        ("group", C.c_int),
+        ("quant_block_q", C.c_int), ("quant_block_k", C.c_int),
+        ("softmax_scale", C.c_float), ("causal", C.c_int),
+        ("out", C.c_void_p), ("lse", C.c_void_p), ("qk_dump", C.c_void_p),
+        ("status", C.c_void_p),
+    ]
+
+
+def library_path() -> Path:
+    return _LIB_PATH
+
+
+def _load() -> C.CDLL:
+    if not _LIB_PATH.exists():
+        raise ImportError(
+            f"{_LIB_PATH} is missing: build the CUDA library with "
+            "`python -m prefill_blockwise_int8_b200.build` (nvcc, sm_100a)")
+    lib = C.CDLL(str(_LIB_PATH))
+    vp, i32 = C.c_void_p, C.c_int
+    lib.tilemix_quantize_blockwise.restype = i32
+    lib.tilemix_quantize_blockwise.argtypes = [
+        vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
+    lib.tilemix_pack_mask.restype = i32
+    lib.tilemix_pack_mask.argtypes = [
+        vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+    lib.tilemix_attn_prefill.restype = i32
+    lib.tilemix_attn_prefill.argtypes = [C.POINTER(AttnParams), vp]
+    lib.tilemix_status_string.restype = C.c_char_p
+    lib.tilemix_status_string.argtypes = [i32]
+    lib.tilemix_last_error.restype = C.c_char_p
+    lib.tilemix_last_error.argtypes = []
+    lib.tilemix_version.restype = C.c_uint32
+    lib.tilemix_version.argtypes = []
+    return lib
+
+
+lib = _load()
+
+
+def tilemix_status_string(status: int) -> str:
+    return lib.tilemix_status_string(status).decode()
+
+
+def tilemix_last_error() -> str:
+    return lib.tilemix_last_error().decode()
+
+
+def tilemix_version() -> int:
+    return int(lib.tilemix_version())
+
+
+# ----------------------------------------------------------------------------
+# torch marshalling
+# ----------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise TilemixError(rc, where, tilemix_last_error())
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dev(t, name, dtype=None):
+    torch = _torch()
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def tilemix_quantize_blockwise(x, cu_seqlens, max_seqlen: int, block: int = 128,
+                               *, x8=None, scale=None, status=None,
+                               stream=None):
+    """Blockwise symmetric INT8 quantisation of fp16 x [T, H, d].
+
+    Returns (x8 int8 [T, H, d], scale fp32 [H, batch, ceil(max_seqlen/block)])."""
+    torch = _torch()
+    _dev(x, "x", torch.float16)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    t, heads, d = x.shape
+    batch = cu_seqlens.numel() - 1
+    nblk = -(-max_seqlen // block)
+    if x8 is None:
+        x8 = torch.empty((t, heads, d), dtype=torch.int8, device=x.device)
+    if scale is None:
+        scale = torch.empty((heads, batch, nblk), dtype=torch.float32,
+                            device=x.device)
+    _dev(x8, "x8", torch.int8)
+    _dev(scale, "scale", torch.float32)
+    _check(lib.tilemix_quantize_blockwise(
+        _ptr(x), _ptr(cu_seqlens), batch, max_seqlen, t, heads, d, block,
+        _ptr(x8), _ptr(scale), _ptr(status), _stream(stream)),
+        "tilemix_quantize_blockwise")
+    return x8, scale
+
+
+def tilemix_pack_mask(route, cu_seqlens, max_seqlen: int, block_m: int,
+                      block_n: int, group: int, *, mask=None, status=None,
+                      stream=None):
+    """uint8 route [B, Hkv, ceil(max_seqlen/block_m), 64] -> uint64 words
+    [B, Hkv, ceil(max_seqlen/block_m)] (returned as torch.int64 storage)."""
+    torch = _torch()
+    _dev(route, "route", torch.uint8)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    batch, hkv, tm, ng = route.shape
+    if ng != 64:
+        raise ValueError("route last dimension must be 64")
+    if mask is None:
+        mask = torch.empty((batch, hkv, tm), dtype=torch.int64,
+                           device=route.device)
+    _dev(mask, "mask")
+    _check(lib.tilemix_pack_mask(
+        _ptr(route), _ptr(cu_seqlens), batch, max_seqlen, hkv, block_m,
+        block_n, group, _ptr(mask), _ptr(status), _stream(stream)),
+        "tilemix_pack_mask")
+    return mask
+
+
+def tilemix_attn_prefill(q, k, v, cu_seqlens, max_seqlen: int, *, q8=None,
+                         q_scale=None, k8=None, k_scale=None, v8=None,
+                         v_scale=None, mask=None, block_m: int = 128,
+                         block_n: int = 128, group: int = 1,
+                         quant_block_q: int = 128, quant_block_k: int = 128,
+                         softmax_scale: float = 0.0, head_map=None,
+                         fp16_only: bool = False, kv_format: int = KV_FP16,
+                         out=None, lse=None, qk_dump=None, status=None,
+                         stream=None):
+    """Causal tile-routed attention.  q fp16 [T, hq, d]; k, v fp16
+    [T, hkv, d] (or k8/v8 int8 + scales with kv_format=KV_INT8).
+    Returns out fp16 [T, hq, d]."""
+    torch = _torch()
+    _dev(q, "q", torch.float16)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    t, hq, d = q.shape
+    kv_src = k8 if kv_format == KV_INT8 else k
+    if kv_src is None:
+        raise ValueError("k (or k8 for KV_INT8) is required")
+    hkv = kv_src.shape[1]
+    for name, tt, dt in (("k", k, torch.float16), ("v", v, torch.float16),
+                         ("q8", q8, torch.int8), ("k8", k8, torch.int8),
+                         ("v8", v8, torch.int8),
+                         ("q_scale", q_scale, torch.float32),
+                         ("k_scale", k_scale, torch.float32),
+                         ("v_scale", v_scale, torch.float32),
+                         ("head_map", head_map, torch.int32),
+                         ("lse", lse, torch.float32),
+                         ("qk_dump", qk_dump, torch.int32)):
+        _dev(tt, name, dt)
+    _dev(mask, "mask")
+    if out is None:
+        out = torch.empty_like(q)
+    _dev(out, "out", torch.float16)
+    p = AttnParams()
+    p.struct_size = C.sizeof(AttnParams)
+    p.kv_format = kv_format
+    p.flags = FLAG_FP16_ONLY if fp16_only else 0
+    p.q, p.q8, p.q_scale = _ptr(q), _ptr(q8), _ptr(q_scale)
+    p.k, p.k8, p.k_scale = _ptr(k), _ptr(k8), _ptr(k_scale)
+    p.v, p.v8, p.v_scale = _ptr(v), _ptr(v8), _ptr(v_scale)
+    p.cu_seqlens = _ptr(cu_seqlens)
+    p.batch = cu_seqlens.numel() - 1
+    p.max_seqlen = max_seqlen
+    p.total_tokens = t
+    p.hq, p.hkv, p.head_dim = hq, hkv, d
+    p.head_map = _ptr(head_map)
+    p.mask = _ptr(mask)
+    p.block_m, p.block_n, p.group = block_m, block_n, group
+    p.quant_block_q, p.quant_block_k = quant_block_q, quant_block_k
+    p.softmax_scale = softmax_scale
+    p.causal = 1
+    p.out, p.lse, p.qk_dump, p.status = (_ptr(out), _ptr(lse), _ptr(qk_dump),
+                                         _ptr(status))
+    _check(lib.tilemix_attn_prefill(C.byref(p), _stream(stream)),
+           "tilemix_attn_prefill")
+    return out

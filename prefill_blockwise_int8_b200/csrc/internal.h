@@ -1,0 +1,71 @@
+// Internal launch interface between the C ABI (tilemix_api.cu) and the
+// kernels.  Not installed, not part of the ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tilemix {
+
+// Device-side status codes (same values as tilemix_status).
+constexpr int kStatusTimeout = 4;
+constexpr int kStatusBadSeqlens = 5;
+
+// Stores `code` into *status if the word is still 0.
+__device__ __forceinline__ void report_status(int32_t* status, int code) {
+  if (status) atomicCAS(reinterpret_cast<int*>(status), 0, code);
+}
+
+cudaError_t launch_quantize_blockwise(const void* x, const int32_t* cu_seqlens,
+                                      int batch, int max_seqlen,
+                                      int total_tokens, int heads,
+                                      int head_dim, int block, int8_t* x8,
+                                      float* scale, int32_t* status,
+                                      cudaStream_t stream);
+
+cudaError_t launch_pack_mask(const uint8_t* route, const int32_t* cu_seqlens,
+                             int batch, int max_seqlen, int hkv, int block_m,
+                             int block_n, int group, uint64_t* mask,
+                             int32_t* status, cudaStream_t stream);
+
+// Everything the fused attention kernel reads.  Passed by value as a
+// __grid_constant__ parameter; the tensor maps must stay 64-byte aligned.
+struct AttnParams {
+  CUtensorMap tm_q;   // fp16 Q  [T, hq, d], box {64, 128, 1}, 128B swizzle
+  CUtensorMap tm_q8;  // int8 Q8 [T, hq, d], box {d, 128, 1}
+  CUtensorMap tm_k;   // fp16 K  [T, hkv, d], box {64, BN, 1}
+  CUtensorMap tm_k8;  // int8 K8 [T, hkv, d], box {d, BN, 1}
+  CUtensorMap tm_v;   // fp16 V  [T, hkv, d], box {64, BN, 1}
+  const int32_t* cu_seqlens;
+  const int32_t* head_map;
+  const uint64_t* mask;
+  const float* q_scale;
+  const float* k_scale;
+  uint16_t* out;     // fp16 bits [T, hq, d]
+  float* lse;
+  int32_t* qk_dump;
+  int32_t* status;
+  int batch, max_seqlen, total_tokens;
+  int hq, hkv, heads_per_kv;
+  int route_bm;      // 64 or 128: query rows per routing word
+  int tm_route;      // ceil(max_seqlen / route_bm)
+  int tn_max;        // ceil(max_seqlen / BN)
+  int group;
+  int quant_block_q, quant_block_k, nbq, nbk;
+  int fp16_only;
+  float scale_log2;  // softmax scale * log2(e)
+};
+
+struct AttnLaunchShape {
+  int head_dim, block_n;
+  bool dual;  // routing rows of 64 inside 128-row compute tiles
+};
+
+cudaError_t launch_attn_prefill(const AttnParams& p, const AttnLaunchShape& s,
+                                cudaStream_t stream);
+
+// Dynamic shared memory and TMEM columns a shape needs (host query).
+int attn_smem_bytes(const AttnLaunchShape& s);
+
+}  // namespace tilemix

@@ -1,0 +1,119 @@
+// Blockwise symmetric INT8 quantiser ("quantize-once") for sm_100a.
+//
+// Method: TileMix (arXiv 2608.17336), paperlayer summary section 3
+// Preliminaries (blockwise quantization, INT8 tensor cores with INT32
+// accumulation) and appendix C Quantization Configuration (Q and K
+// quantised blockwise and symmetrically once per attention call).
+// Per (sequence, head, block of tokens): scale = absmax / 127 (IEEE fp32
+// division), code = clamp(round_half_even(x / scale), -127, 127).
+//
+// HBM-bound: one CTA reads one block (up to 32 KB of fp16) once into
+// registers with 16-byte loads, reduces the absmax, and writes the codes
+// with 8-byte stores.  Rows of a block are strided by heads * d in memory,
+// each row contiguous.
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+namespace tilemix {
+namespace {
+
+constexpr int kQThreads = 256;
+constexpr int kMaxVecs = 16;  // 16-byte vectors per thread: block*d <= 32768
+
+__global__ void __launch_bounds__(kQThreads)
+    quantize_kernel(const __half* __restrict__ x,
+                    const int32_t* __restrict__ cu_seqlens, int batch,
+                    int max_seqlen, int total_tokens, int heads, int d,
+                    int block, int nblk, int8_t* __restrict__ x8,
+                    float* __restrict__ scale, int32_t* status) {
+  const int t = blockIdx.x;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int start = cu_seqlens[b];
+  const int len = cu_seqlens[b + 1] - start;
+  if (start < 0 || len < 0 || len > max_seqlen || start + len > total_tokens) {
+    if (threadIdx.x == 0) report_status(status, kStatusBadSeqlens);
+    return;
+  }
+  float* s_out = scale + (static_cast<size_t>(h) * batch + b) * nblk + t;
+  const int r0 = t * block;
+  if (r0 >= len) {
+    if (threadIdx.x == 0) *s_out = 0.0f;
+    return;
+  }
+  const int rows = min(block, len - r0);
+  const int vpr = d / 8;  // 8 halves per 16-byte vector
+  const int nv = rows * vpr;
+  const size_t row_stride = static_cast<size_t>(heads) * d;
+  const __half* base = x + (static_cast<size_t>(start + r0) * heads + h) * d;
+
+  uint4 v[kMaxVecs];
+  __half2 amax2 = __float2half2_rn(0.0f);
+#pragma unroll
+  for (int k = 0; k < kMaxVecs; ++k) {
+    const int idx = threadIdx.x + k * kQThreads;
+    if (idx < nv) {
+      const int r = idx / vpr;
+      const int c = idx - r * vpr;
+      v[k] = __ldg(reinterpret_cast<const uint4*>(base + r * row_stride) + c);
+      const __half2* hv = reinterpret_cast<const __half2*>(&v[k]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) amax2 = __hmax2(amax2, __habs2(hv[e]));
+    }
+  }
+  float amax = fmaxf(__low2float(amax2), __high2float(amax2));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  __shared__ float warp_max[kQThreads / 32];
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = warp_max[0];
+#pragma unroll
+  for (int w = 1; w < kQThreads / 32; ++w) amax = fmaxf(amax, warp_max[w]);
+
+  const float s = __fdiv_rn(amax, 127.0f);
+  if (threadIdx.x == 0) *s_out = s;
+  int8_t* qbase = x8 + (static_cast<size_t>(start + r0) * heads + h) * d;
+#pragma unroll
+  for (int k = 0; k < kMaxVecs; ++k) {
+    const int idx = threadIdx.x + k * kQThreads;
+    if (idx < nv) {
+      const int r = idx / vpr;
+      const int c = idx - r * vpr;
+      const __half* hv = reinterpret_cast<const __half*>(&v[k]);
+      uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        int q = 0;
+        if (amax != 0.0f) {
+          q = __float2int_rn(__fdiv_rn(__half2float(hv[e]), s));
+          q = max(-127, min(127, q));
+        }
+        packed[e >> 2] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (e & 3));
+      }
+      *reinterpret_cast<uint2*>(qbase + r * row_stride + c * 8) =
+          make_uint2(packed[0], packed[1]);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_blockwise(const void* x, const int32_t* cu_seqlens,
+                                      int batch, int max_seqlen,
+                                      int total_tokens, int heads,
+                                      int head_dim, int block, int8_t* x8,
+                                      float* scale, int32_t* status,
+                                      cudaStream_t stream) {
+  const int nblk = (max_seqlen + block - 1) / block;
+  dim3 grid(nblk, heads, batch);
+  quantize_kernel<<<grid, kQThreads, 0, stream>>>(
+      static_cast<const __half*>(x), cu_seqlens, batch, max_seqlen,
+      total_tokens, heads, head_dim, block, nblk, x8, scale, status);
+  return cudaGetLastError();
+}
+
+}  // namespace tilemix

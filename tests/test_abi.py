@@ -1,0 +1,142 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/tilemix.h declares, the Python struct mirrors the C layout, and the
+host-side argument checks reject bad calls before any launch."""
+import ctypes as C
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tilemix.h")
+
+tm = pytest.importorskip("prefill_blockwise_int8_b200")
+
+OK, INVALID, UNSUPPORTED, NO_DEVICE = 0, 1, 2, 6
+FAKE = 0x10000  # 64 KiB: 16-byte aligned, never dereferenced on the host
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tilemix_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declarations_are_exported():
+    names = declared_functions()
+    assert set(names) == set(tm.EXPORTED_SYMBOLS)
+    for n in names:
+        assert hasattr(tm.lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", str(tm.library_path())],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (tilemix_\w+)", out))
+    assert set(names) <= exported
+
+
+def test_version_and_status_strings():
+    assert tm.tilemix_version() >> 16 == 1
+    for code in range(7):
+        assert tm.tilemix_status_string(code)
+    assert tm.tilemix_status_string(99) == "unknown status"
+
+
+def test_params_struct_layout_matches_c():
+    fields = [f for f, _ in tm.AttnParams._fields_]
+    prog = ["#include <stdio.h>", "#include <stddef.h>", '#include "tilemix.h"',
+            "int main(void) {",
+            'printf("size %zu\\n", sizeof(tilemix_attn_params));']
+    for f in fields:
+        prog.append(f'printf("{f} %zu\\n", offsetof(tilemix_attn_params, {f}));')
+    prog.append("return 0; }")
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "layout.c")
+        exe = os.path.join(d, "layout")
+        open(c, "w").write("\n".join(prog))
+        subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I",
+                        os.path.join(ROOT, "include"), c, "-o", exe],
+                       check=True)
+        out = subprocess.run([exe], capture_output=True, text=True,
+                             check=True).stdout
+    got = dict(line.split() for line in out.strip().splitlines())
+    assert int(got["size"]) == C.sizeof(tm.AttnParams)
+    for f in fields:
+        assert int(got[f]) == getattr(tm.AttnParams, f).offset, f
+
+
+def good_params(**kw):
+    p = tm.AttnParams()
+    p.struct_size = C.sizeof(tm.AttnParams)
+    p.kv_format = tm.KV_FP16
+    p.q = p.k = p.v = p.out = p.q8 = p.k8 = FAKE
+    p.q_scale = p.k_scale = p.cu_seqlens = p.mask = FAKE
+    p.batch, p.max_seqlen, p.total_tokens = 2, 4096, 8192
+    p.hq, p.hkv, p.head_dim = 24, 8, 128
+    p.block_m, p.block_n, p.group = 128, 64, 1
+    p.causal = 1
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def call(p):
+    return tm.lib.tilemix_attn_prefill(C.byref(p), None)
+
+
+def test_attn_host_checks_accept_a_valid_call():
+    # valid arguments get past every host check; with no GPU in this
+    # process the call then stops at the device check
+    rc = call(good_params())
+    assert rc in (NO_DEVICE, OK), tm.tilemix_last_error()
+
+
+@pytest.mark.parametrize("field,value,expect", [
+    ("struct_size", 8, INVALID),
+    ("causal", 0, UNSUPPORTED),
+    ("head_dim", 96, UNSUPPORTED),
+    ("block_n", 32, UNSUPPORTED),
+    ("block_m", 256, UNSUPPORTED),
+    ("kv_format", 7, INVALID),
+    ("group", 0, INVALID),
+    ("hkv", 5, INVALID),              # 24 % 5 != 0 and no head_map
+    ("max_seqlen", 64 * 64 + 1, INVALID),   # 65 key tiles of 64 with g = 1
+    ("q", 0, INVALID),
+    ("out", FAKE + 8, INVALID),       # misaligned for TMA
+    ("mask", 0, INVALID),             # routed mode needs the words
+    ("quant_block_k", 96, UNSUPPORTED),     # not a multiple of block_n
+    ("flags", 0x80, INVALID),
+])
+def test_attn_host_checks_reject(field, value, expect):
+    assert call(good_params(**{field: value})) == expect
+    assert tm.tilemix_last_error()
+
+
+def test_attn_block_m64_needs_block_n64():
+    assert call(good_params(block_m=64, block_n=128)) == UNSUPPORTED
+
+
+def test_attn_fp16_only_needs_no_int8_operands():
+    p = good_params(flags=tm.FLAG_FP16_ONLY, mask=0, q8=0, k8=0, q_scale=0,
+                    k_scale=0)
+    assert call(p) in (NO_DEVICE, OK)
+
+
+def test_group_lifts_the_64_bit_limit():
+    p = good_params(max_seqlen=64 * 64 * 2, total_tokens=64 * 64 * 4, group=2)
+    assert call(p) in (NO_DEVICE, OK)
+
+
+def test_quantize_and_pack_host_checks():
+    q = tm.lib.tilemix_quantize_blockwise
+    assert q(None, FAKE, 1, 128, 128, 2, 64, 128, FAKE, FAKE, None, None) == INVALID
+    assert q(FAKE, FAKE, 1, 128, 128, 2, 60, 128, FAKE, FAKE, None, None) == INVALID
+    assert q(FAKE, FAKE, 1, 128, 128, 2, 256, 256, FAKE, FAKE, None, None) == INVALID
+    assert q(FAKE + 4, FAKE, 1, 128, 128, 2, 64, 128, FAKE, FAKE, None, None) == INVALID
+    assert q(FAKE, FAKE, 1, 128, 128, 2, 64, 128, FAKE, FAKE, None, None) in (NO_DEVICE, OK)
+    assert q(FAKE, FAKE, 0, 0, 0, 2, 64, 128, FAKE, FAKE, None, None) == OK
+    pk = tm.lib.tilemix_pack_mask
+    assert pk(FAKE, FAKE, 1, 64 * 65, 1, 64, 64, 1, FAKE, None, None) == INVALID
+    assert pk(FAKE, FAKE, 1, 64 * 65, 1, 64, 64, 2, FAKE, None, None) in (NO_DEVICE, OK)
+    assert pk(FAKE + 8, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
+    assert pk(None, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID

@@ -1,0 +1,275 @@
+"""GPU parity: every CUDA step against the CPU oracle on the same seeded
+inputs, through the C ABI.
+
+* quantiser: Q8/K8 codes and fp32 scales byte-exact;
+* packer: routing words bit-exact (junk in illegal groups cleared);
+* attention: INT32 score tiles of INT8-routed groups bit-exact; fp16 output
+  within max-abs 3e-3 and relative L2 2e-3 of the fp64 oracle; LSE within
+  1e-3; at sizes that span several tiles with ragged tails, and at the full
+  workload sizes on sampled rows.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+from _gpu_path import (LSE_ABS, compare, dev_tensor, run_gpu, run_oracle,
+                       sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def tm():
+    import prefill_blockwise_int8_b200 as m
+    return m
+
+
+def small(L, *, hq=4, hkv=2, d=128, bm=128, bn=64, g=1, recipe="diag_first",
+          cov=0.75, seed=5, outliers=True, qb=128, kb=128):
+    lens = [L] if isinstance(L, int) else list(L)
+    w = W.Workload(name="small", batch=len(lens), hq=hq, hkv=hkv, d=d,
+                   block_m=bm, block_n=bn, group=g, seqlen=0, outliers=outliers,
+                   mask_recipe=recipe, coverage=cov, seed=seed,
+                   mask_seed=seed + 100, quant_block_q=qb, quant_block_k=kb,
+                   coverage_unit="kv_head")
+    lens = np.array(lens, dtype=np.int32)
+    # the fixed-length generator stream, drawn for T = sum(lens) tokens
+    q, k, v = W.qkv(w.with_(seqlen=1), lens)
+    return dict(workload=w, seqlens=lens, cu_seqlens=W.cu_seqlens(lens),
+                max_seqlen=int(max(lens.max(), 1)), group=g, q=q, k=k, v=v,
+                route=W.route_bytes(w, lens))
+
+
+# ----------------------------------------------------------------------------
+# quantiser and packer
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("block", [64, 128])
+def test_quantize_bitexact_varlen(tm, d, block):
+    lens = np.array([1, 127, 128, 129, 300, 0, 1000], dtype=np.int32)
+    cu = W.cu_seqlens(lens)
+    rng = np.random.default_rng(d + block)
+    x = (rng.standard_normal((lens.sum(), 3, d)) * 4).astype(np.float16)
+    x[cu[3]:cu[3] + 5, 2, 7] = 300.0   # an outlier
+    x[cu[2]:cu[3], 1, :] = 0           # an all-zero block
+    ref8, refs = oracle.quantize_blockwise(x, cu, int(lens.max()), block)
+    g8, gs = tm.tilemix_quantize_blockwise(dev_tensor(x), dev_tensor(cu),
+                                           int(lens.max()), block)
+    torch.cuda.synchronize()
+    assert np.array_equal(g8.cpu().numpy(), ref8)
+    assert np.array_equal(gs.cpu().numpy().view(np.uint32), refs.view(np.uint32))
+
+
+def test_quantize_golden_ties(tm):
+    here = os.path.dirname(__file__)
+    cases = json.load(open(os.path.join(here, "golden",
+                                        "quantize_examples.json")))["cases"]
+    for c in cases:
+        x = np.array(c["x"], dtype=np.float16)
+        L, d = x.shape
+        xp = np.zeros((L, 1, 8), dtype=np.float16)  # head_dim multiple of 8
+        xp[:, 0, :d] = x
+        g8, gs = tm.tilemix_quantize_blockwise(
+            dev_tensor(xp), dev_tensor(np.array([0, L], np.int32)), L, L)
+        torch.cuda.synchronize()
+        assert gs.item() == np.float32(c["scale"]), c["name"]
+        assert np.array_equal(g8.cpu().numpy()[:, 0, :d], np.array(c["q"])), c["name"]
+
+
+def test_pack_bitexact_all_workloads(tm):
+    for w in [W.TINY, W.LLAMA32_3B_4K, W.VARLEN16, W.INT8KV_16K,
+              W.sweep_32k(75)]:
+        lens = W.seqlens(w)
+        cu = W.cu_seqlens(lens)
+        g = W.group_size(w, lens)
+        route = W.route_bytes(w, lens, junk_in_illegal=True)
+        ref = oracle.pack_mask(route, cu, int(lens.max()), w.block_m,
+                               w.block_n, g)
+        got = tm.tilemix_pack_mask(dev_tensor(route), dev_tensor(cu),
+                                   int(lens.max()), w.block_m, w.block_n, g)
+        torch.cuda.synchronize()
+        assert np.array_equal(got.cpu().numpy().view(np.uint64), ref), w.name
+
+
+# ----------------------------------------------------------------------------
+# attention, small sizes, every output element
+# ----------------------------------------------------------------------------
+
+def test_tiny_workload_full(tm):
+    inp = W.make(W.TINY)
+    got = run_gpu(inp, want_lse=True, want_dump=True)
+    assert got["status"] == 0
+    (ref, lse), kw = run_oracle(inp, want_lse=True)
+    assert np.array_equal(got["q8"], kw["q8"])
+    assert np.array_equal(got["mask"], kw["mask"])
+    compare(got["out"], ref)
+    assert np.abs(got["lse"] - lse).max() <= LSE_ABS
+    dump = oracle.qk_dump(inp["cu_seqlens"], 256, kw["q8"], kw["k8"],
+                          kw["mask"], hq=2, hkv=1, d=64, block_m=64,
+                          block_n=64, group=1, fill=-1)
+    assert np.array_equal(got["dump"], dump)
+    assert (dump != -1).any()
+
+
+CASES = {
+    # name: (lens, kwargs of small())
+    "d128_bn64_ragged": ([1000], dict()),
+    "d128_bn128_two_seqs": ([700, 300], dict(bn=128, hkv=1, recipe="exact", cov=0.5)),
+    "d64_bn128_g2": ([1100, 257], dict(d=64, bn=128, g=2, recipe="exact", cov=0.5)),
+    "d64_bm64_dual": ([700], dict(d=64, bm=64, bn=64, recipe="bernoulli", cov=0.5)),
+    "d128_bm64_dual": ([513, 64, 200], dict(bm=64, bn=64, recipe="bernoulli", cov=0.5)),
+    "mha": ([333], dict(hq=3, hkv=3, recipe="exact", cov=0.5)),
+    "gqa7": ([520], dict(hq=7, hkv=1, recipe="exact", cov=0.5)),
+    "all_int8": ([600], dict(recipe="exact", cov=1.0)),
+    "all_fp16_mask": ([600], dict(recipe="exact", cov=0.0)),
+    "no_outliers": ([400, 1], dict(outliers=False, recipe="bernoulli", cov=0.5)),
+    "qblock64_kblock64": ([450], dict(qb=64, kb=64, recipe="exact", cov=0.5)),
+    "kblock256_bn128": ([700], dict(bn=128, kb=256, qb=256, recipe="exact", cov=0.5)),
+    "seq_len_one": ([1], dict()),
+    "tiny_seqs_and_empty": ([1, 2, 0, 3, 130], dict(recipe="bernoulli", cov=0.5)),
+    "exactly_64_groups": ([4096], dict(hq=2, hkv=1, recipe="exact", cov=0.5)),
+    "exactly_64_groups_g2": ([8192], dict(hq=1, hkv=1, bn=64, g=2, recipe="exact", cov=0.5)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_attention_small_cases(tm, name):
+    lens, kw = CASES[name]
+    inp = small(lens, **kw)
+    got = run_gpu(inp, want_lse=True)
+    assert got["status"] == 0
+    work = sum(int(L) * int(L) for L in lens) * inp["workload"].hq
+    # every row while the oracle stays within a few seconds, else a sample
+    rows = None if work <= 8_000_000 else sample_rows(
+        inp["seqlens"], inp["cu_seqlens"], per_seq=64,
+        block=inp["workload"].block_m)
+    (ref, lse), okw = run_oracle(inp, want_lse=True, rows=rows)
+    assert np.array_equal(got["q8"], okw["q8"])
+    assert np.array_equal(got["k8"], okw["k8"])
+    compare(got["out"], ref, rows=rows)
+    sel = slice(None) if rows is None else rows
+    assert np.abs(got["lse"][:, sel] - lse[:, sel]).max() <= LSE_ABS
+
+
+def test_fp16_only_flag(tm):
+    inp = small([900], recipe="exact", cov=1.0)
+    got = run_gpu(inp, fp16_only=True)
+    ref, _ = run_oracle(inp, fp16_only=True)
+    compare(got["out"], ref)
+    # the flag ignores the mask: all-INT8 words must not change the result
+    ref_int8, _ = run_oracle(inp)
+    assert np.abs(ref_int8 - ref).max() > 1e-3
+
+
+def test_explicit_head_map(tm):
+    inp = small([640], hq=4, hkv=2, recipe="exact", cov=0.5)
+    hm = [1, 0, 1, 0]
+    got = run_gpu(inp, head_map=hm)
+    ref, _ = run_oracle(inp, head_map=hm)
+    compare(got["out"], ref)
+
+
+def test_int8_tiles_bitexact_dump(tm):
+    inp = small([700, 300], bm=128, bn=128, hkv=1, recipe="exact", cov=0.5)
+    got = run_gpu(inp, want_dump=True)
+    _, kw = run_oracle(inp, rows=np.array([0]))
+    dump = oracle.qk_dump(inp["cu_seqlens"], 700, kw["q8"], kw["k8"],
+                          kw["mask"], hq=4, hkv=1, d=128, block_m=128,
+                          block_n=128, group=1, fill=-1)
+    assert np.array_equal(got["dump"], dump)
+
+
+def test_garbage_bits_in_illegal_groups_change_nothing(tm):
+    inp = small([777, 200], bm=128, bn=64, recipe="exact", cov=0.5)
+    clean = run_gpu(inp)["out"]
+    w = inp["workload"]
+    junk = W.route_bytes(w, inp["seqlens"], junk_in_illegal=True)
+    dirty = run_gpu(inp, route=junk)["out"]
+    assert np.array_equal(clean, dirty)
+
+
+def test_deterministic_and_stream(tm):
+    inp = small([1000], recipe="exact", cov=0.5)
+    a = run_gpu(inp)["out"]
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b = run_gpu(inp, stream=s)["out"]
+    assert np.array_equal(a, b)
+
+
+def test_coverage_changes_result_monotonically(tm):
+    # more INT8 coverage moves the output further from the all-FP16 result
+    inp = small([1024], recipe="exact", cov=0.0)
+    base = run_gpu(inp, fp16_only=True)["out"]
+    devs = []
+    for cov in (0.0, 0.5, 1.0):
+        inp2 = small([1024], recipe="exact", cov=cov)
+        devs.append(np.abs(run_gpu(inp2)["out"] - base).mean())
+    assert devs[0] == 0.0
+    assert devs[0] < devs[1] < devs[2]
+
+
+# ----------------------------------------------------------------------------
+# device-detected errors
+# ----------------------------------------------------------------------------
+
+def test_bad_cu_seqlens_sets_status(tm):
+    inp = small([300, 200])
+    cu = np.array([0, 400, 500], np.int32)   # length 400 > max_seqlen 300
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q = dev_tensor(inp["q"])
+    k = dev_tensor(inp["k"])
+    v = dev_tensor(inp["v"])
+    tm.tilemix_attn_prefill(q, k, v, dev_tensor(cu), 300, fp16_only=True,
+                            block_m=128, block_n=64, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 5
+
+
+def test_head_map_out_of_range_sets_status(tm):
+    inp = small([300])
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tm.tilemix_attn_prefill(
+        dev_tensor(inp["q"]), dev_tensor(inp["k"]), dev_tensor(inp["v"]),
+        dev_tensor(inp["cu_seqlens"]), 300, fp16_only=True, block_m=128,
+        block_n=64, head_map=dev_tensor(np.array([0, 1, 2, 0], np.int32)),
+        status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 5
+
+
+def test_int8_kv_format_reports_unsupported_until_built(tm):
+    inp = small([128])
+    with pytest.raises(tm.TilemixError):
+        tm.tilemix_attn_prefill(dev_tensor(inp["q"]), None, None,
+                                dev_tensor(inp["cu_seqlens"]), 128,
+                                k8=dev_tensor(np.zeros((128, 2, 128), np.int8)),
+                                kv_format=tm.KV_INT8)
+
+
+# ----------------------------------------------------------------------------
+# full workload sizes, sampled rows
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("wname", [
+    W.LLAMA32_3B_4K.name, W.VARLEN16.name, W.sweep_32k(75).name,
+    W.sweep_32k(0).name, W.sweep_32k(100).name])
+def test_full_size_sampled_rows(tm, wname):
+    w = W.WORKLOADS[wname]
+    inp = W.make(w)
+    got = run_gpu(inp)
+    assert got["status"] == 0
+    rows = sample_rows(inp["seqlens"], inp["cu_seqlens"], per_seq=16,
+                       block=w.block_m)
+    ref, kw = run_oracle(inp, rows=rows)
+    assert np.array_equal(got["q8"], kw["q8"])
+    assert np.array_equal(got["sq"].view(np.uint32), kw["q_scale"].view(np.uint32))
+    assert np.array_equal(got["mask"], kw["mask"])
+    compare(got["out"], ref, rows=rows)
