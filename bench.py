@@ -1,0 +1,467 @@
+#!/usr/bin/env python
+"""Throughput of tile-routed FP16/INT8 causal prefill attention on B200.
+
+One step = the whole hot path on one batch of synthetic inputs resident in
+HBM: blockwise INT8 quantisation of Q and of K, packing of the routing
+words, and the fused attention kernel.  Reported:
+
+  value       tokens/s of the step (all ranks; weak scaling: every rank runs
+              its own replica of the workload, no collective on the data path)
+  effective   4 * d * Hq * sum L(L+1)/2 FLOP per step / step time
+  roofline    the attention kernel against the mixed FP16/INT8 tensor-core
+              roofline t_roof = (QK_fp16 + PV) / P_fp16 + QK_int8 / P_int8
+  e2e         the same metric through the public API with host buffers:
+              pinned host -> device copies of Q, K, V and the routing bytes and
+              the device -> host copy of the output inside the timed region
+  cpu_baseline  the CPU oracle, timed on this host's cores on a bounded
+              sample of the same workload (rank 0, one GPU only)
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU oracle as the reference arm
+
+L2 is flushed (a 256 MiB write) before every timed step, outside the
+per-step CUDA events.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "prefill attn tokens/s & effective TFLOPS vs mixed FP16/INT8 roofline"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = W.LLAMA32_3B_4K.name
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                  "bf16_tflops_sustained": 1400.0}
+INT8_OVER_FP16 = 2.0  # nominal dense INT8 / FP16 tensor ratio (4.5 / 2.25 P)
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["tilemix", "reference"],
+                    default="tilemix")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(W.WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return args
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(w, inp, share):
+    lens = inp["seqlens"]
+    return {
+        "workload": w.name,
+        "batch": int(len(lens)),
+        "seq_len": int(lens.max()) if w.seqlen == 0 else int(w.seqlen),
+        "total_tokens": int(lens.sum()),
+        "hq": w.hq, "hkv": w.hkv, "head_dim": w.d,
+        "tile": f"{w.block_m}x{w.block_n}", "group": int(inp["group"]),
+        "kv_format": w.kv_format,
+        "int8_group_coverage": w.coverage,
+        "int8_pair_share": round(share, 4),
+        "quant_block": [w.quant_block_q, w.quant_block_k],
+        "inputs": "N(0,1) fp16" + (", 4 outlier channels x20 per Q/K head"
+                                    if w.outliers else ""),
+        "parallelism": "replicas",
+        "l2": "flushed (256 MiB write) before every timed step",
+    }
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle legs
+# ----------------------------------------------------------------------------
+
+def oracle_sample_rate(inp, target_s, seed=7):
+    """tokens/s of the oracle on uniformly drawn query rows (all heads, the
+    full causal row each).  Returns (tokens/s, sample description, cores)."""
+    import oracle
+    args, kw = oracle.prepare(inp)
+    total = int(inp["seqlens"].sum())
+    rng = np.random.default_rng(seed)
+    n = 16
+    elapsed = 0.0
+    done = 0
+    while True:
+        rows = np.sort(rng.choice(total, size=min(n, total), replace=False))
+        t0 = time.perf_counter()
+        oracle.attn_prefill(*args, rows=rows, **kw)
+        dt = time.perf_counter() - t0
+        elapsed += dt
+        done += len(rows)
+        if elapsed >= target_s or done >= total:
+            break
+        per_row = elapsed / done
+        n = int(max(16, min(total, (target_s - elapsed) / per_row)))
+    cores = os.cpu_count() or 1
+    desc = (f"{done} query tokens drawn uniformly from {total} "
+            f"(all {inp['workload'].hq} heads, full causal rows), "
+            f"{elapsed:.1f} s on {cores} threads; oracle quantiser and "
+            f"packer excluded")
+    return done / elapsed, desc, cores
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = W.WORKLOADS[args.workload]
+    inp = W.make(w)
+    share = None
+    import oracle
+    oargs, kw = oracle.prepare(inp)
+    total = int(inp["seqlens"].sum())
+    budget = 150.0  # seconds for warmup + steps together
+    per_step = budget / (args.steps + args.warmup)
+    rng = np.random.default_rng(11)
+    # calibrate rows per step
+    rows = np.sort(rng.choice(total, size=16, replace=False))
+    t0 = time.perf_counter()
+    oracle.attn_prefill(*oargs, rows=rows, **kw)
+    per_row = (time.perf_counter() - t0) / 16
+    n = int(max(1, min(total, per_step / per_row)))
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(total, size=n, replace=False))
+        t0 = time.perf_counter()
+        oracle.attn_prefill(*oargs, rows=rows, **kw)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    value = n * len(times) / sum(times)
+    cores = os.cpu_count() or 1
+    fp16_pairs, int8_pairs = _pairs(inp, oracle.pack_mask(
+        inp["route"], inp["cu_seqlens"], inp["max_seqlen"], w.block_m,
+        w.block_n, inp["group"]))
+    share = int8_pairs / (fp16_pairs + int8_pairs)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, inp, share),
+        "cpu_baseline": {
+            "value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"each step {n} query tokens drawn uniformly from {total}"
+                      f" (all heads, full causal rows) on {cores} threads"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _pairs(inp, mask_words):
+    from prefill_blockwise_int8_b200.roofline import pair_counts
+    w = inp["workload"]
+    return pair_counts(inp["seqlens"], mask_words, w.block_m, w.block_n,
+                       inp["group"], w.hq, w.hkv)
+
+
+# ----------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        import tempfile
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv",
+                                               delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200", "-i",
+                 str(self.dev)], stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.out.flush()
+
+    def summary(self):
+        try:
+            lines = open(self.out.name).read().strip().splitlines()
+        except OSError:
+            lines = []
+        finally:
+            try:
+                os.unlink(self.out.name)
+            except OSError:
+                pass
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for ln in lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=datetime.timedelta(seconds=300))
+
+    import prefill_blockwise_int8_b200 as tm
+
+    w = W.WORKLOADS[args.workload]
+    inp = W.make(w)
+    lens, cu_np = inp["seqlens"], inp["cu_seqlens"]
+    ms, g = inp["max_seqlen"], inp["group"]
+    T = int(lens.sum())
+    t_h = {k: torch.from_numpy(inp[k]) for k in ("q", "k", "v", "route")}
+    cu_h = torch.from_numpy(cu_np)
+    q = t_h["q"].to(dev)
+    k = t_h["k"].to(dev)
+    v = t_h["v"].to(dev)
+    route = t_h["route"].to(dev)
+    cu = cu_h.to(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    q8 = torch.empty((T, w.hq, w.d), dtype=torch.int8, device=dev)
+    k8 = torch.empty((T, w.hkv, w.d), dtype=torch.int8, device=dev)
+    sq = torch.empty((w.hq, len(lens), -(-ms // w.quant_block_q)),
+                     dtype=torch.float32, device=dev)
+    sk = torch.empty((w.hkv, len(lens), -(-ms // w.quant_block_k)),
+                     dtype=torch.float32, device=dev)
+    mask = torch.empty(route.shape[:3], dtype=torch.int64, device=dev)
+    out = torch.empty_like(q)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 4
+
+    def step(attn_events=None):
+        tm.tilemix_quantize_blockwise(q, cu, ms, w.quant_block_q, x8=q8,
+                                      scale=sq, status=status)
+        tm.tilemix_quantize_blockwise(k, cu, ms, w.quant_block_k, x8=k8,
+                                      scale=sk, status=status)
+        tm.tilemix_pack_mask(route, cu, ms, w.block_m, w.block_n, g, mask=mask,
+                             status=status)
+        if attn_events:
+            attn_events[0].record(stream)
+        tm.tilemix_attn_prefill(
+            q, k, v, cu, ms, q8=q8, q_scale=sq, k8=k8, k_scale=sk, mask=mask,
+            block_m=w.block_m, block_n=w.block_n, group=g,
+            quant_block_q=w.quant_block_q, quant_block_k=w.quant_block_k,
+            out=out, status=status)
+        if attn_events:
+            attn_events[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()} during warmup")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
+          for _ in range(args.steps)]
+    smi_index = local
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        parts = [p.strip() for p in vis.split(",")]
+        if local < len(parts):
+            smi_index = parts[local]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(smi_index) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step((ev[i][1], ev[i][2]))
+            ev[i][3].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()} in timed region")
+    ms_step = total_ms / args.steps
+    value = world * T / (ms_step * 1e-3)
+
+    # ---- e2e through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        pin = {kk: t.pin_memory() for kk, t in t_h.items()}
+        cu_pin = cu_h.pin_memory()
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        n_e2e = max(3, min(args.steps, 8))
+        ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+              for _ in range(n_e2e)]
+        h2d = sum(t.numel() * t.element_size() for t in pin.values()) + \
+            cu_pin.numel() * 4
+        d2h = out_h.numel() * out_h.element_size()
+
+        def e2e_step():
+            q.copy_(pin["q"], non_blocking=True)
+            k.copy_(pin["k"], non_blocking=True)
+            v.copy_(pin["v"], non_blocking=True)
+            route.copy_(pin["route"], non_blocking=True)
+            cu.copy_(cu_pin, non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        for i in range(n_e2e):
+            flush.zero_()
+            ee[i][0].record(stream)
+            e2e_step()
+            ee[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = sum(a.elapsed_time(b) for a, b in ee)
+        if world > 1:
+            tt = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": world * T / (e_ms / n_e2e * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": n_e2e}
+
+    # ---- roofline of the attention kernel ----
+    from prefill_blockwise_int8_b200 import roofline as R
+    mask_np = mask.cpu().numpy().view(np.uint64)
+    fp16_pairs, int8_pairs = R.pair_counts(lens, mask_np, w.block_m,
+                                           w.block_n, g, w.hq, w.hkv)
+    wk = R.work(lens, w.d, w.hq, fp16_pairs, int8_pairs)
+    peaks, peak_src = load_peaks()
+    p16 = float(peaks["bf16_tflops"]) * 1e12  # fp16 dense = bf16 dense rate
+    p8 = p16 * INT8_OVER_FP16
+    t_roof = R.roofline_seconds(wk, p16, p8)
+    attn_s = statistics.mean(attn_ms) * 1e-3
+    achieved = wk["effective"] / attn_s / 1e12
+    peak_eff = wk["effective"] / t_roof / 1e12
+    roof = {
+        "bound": "tensor", "achieved": round(achieved, 2),
+        "peak": round(peak_eff, 2), "unit": "TFLOP/s",
+        "frac": round(achieved / peak_eff, 4), "traffic": None,
+        "kernel": "attn_fwd_kernel",
+        "attn_ms": round(attn_s * 1e3, 4),
+        "t_roof_ms": round(t_roof * 1e3, 4),
+        "peak_basis": (f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s"
+                       f" for FP16; INT8 = x{INT8_OVER_FP16:g} (nominal "
+                       "4.5/2.25 P dense ratio); mixed by routed pair share "
+                       f"{wk['int8_pair_share']:.4f}"),
+        "algorithmic_flop_per_launch": wk["effective"],
+        "hbm_bytes_min_per_launch": R.min_hbm_bytes(
+            T, w.hq, w.hkv, w.d, wk["int8_pair_share"]),
+    }
+
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        rate, desc, cores = oracle_sample_rate(inp, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": desc}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp16+int8", "data": "synthetic",
+        "config": workload_config(w, inp, wk["int8_pair_share"]),
+        "effective_tflops": wk["effective"] / (ms_step * 1e-3) / 1e12 * world,
+        "attn_effective_tflops": achieved,
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

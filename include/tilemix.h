@@ -173,8 +173,9 @@ typedef struct {
   float* lse;                /* optional dev fp32 [hq, T]: natural-log LSE  */
   /* Optional debug output, dev int32 [batch, hq, Tm_max, Tn_max, block_m,
    * block_n] with Tn_max = ceil(max_seqlen / block_n): the raw INT32
-   * accumulators of every INT8-routed legal tile, written for rows inside
-   * the sequence; entries of other tiles are left untouched. */
+   * accumulators of every INT8-routed legal tile, causally masked positions
+   * included, written for the rows and keys inside the sequence; every other
+   * entry is left untouched. */
   int32_t* qk_dump;
   int32_t* status;           /* optional dev int32, see above               */
 } tilemix_attn_params;

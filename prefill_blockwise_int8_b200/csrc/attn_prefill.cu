@@ -387,7 +387,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                  p.route_bm +
              rr) *
                 BN;
-        for (int j = 0; j < BN; ++j) dst[j] = static_cast<int32_t>(sv[j]);
+        const int keys_left = len - n * BN;  // keys inside the sequence
+        for (int j = 0; j < BN; ++j)
+          if (j < keys_left) dst[j] = static_cast<int32_t>(sv[j]);
       }
 
       // Scores in log2 units are x_j = S_j * c with c > 0 (or 0 for an
