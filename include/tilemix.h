@@ -174,8 +174,9 @@ typedef struct {
   /* Optional debug output, dev int32 [batch, hq, Tm_max, Tn_max, block_m,
    * block_n] with Tn_max = ceil(max_seqlen / block_n): the raw INT32
    * accumulators of every INT8-routed legal tile, causally masked positions
-   * included, written for the rows and keys inside the sequence; every other
-   * entry is left untouched. */
+   * included, written for the rows and keys inside the sequence.  Keys past
+   * the last query row of the routing row (masked for all of its rows) may be
+   * skipped in 64-key steps; every other entry is left untouched. */
   int32_t* qk_dump;
   int32_t* status;           /* optional dev int32, see above               */
 } tilemix_attn_params;

@@ -283,6 +283,19 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Exact INT32 -> FP32 for |v| < 2^22 without the conversion unit:
+// 0x4B400000 is 1.5 * 2^23; adding v to its bit pattern gives the float
+// 1.5 * 2^23 + v exactly, and subtracting 1.5 * 2^23 (see int_bias_f32)
+// leaves v.  The caller does the subtraction (two at a time).
+constexpr uint32_t kIntBiasBits = 0x4B400000u;
+constexpr float kIntBias = 12582912.0f;  // 1.5 * 2^23
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);  // .x (low 16 bits) = lo
   return *reinterpret_cast<uint32_t*>(&h);

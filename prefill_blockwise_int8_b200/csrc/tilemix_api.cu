@@ -213,7 +213,7 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
                 "attn: hq %d not a multiple of hkv %d and no head_map", a->hq,
                 a->hkv);
   if (a->hq > 65535 || a->batch > 65535 ||
-      (a->max_seqlen + 127) / 128 > 65535)
+      (a->max_seqlen + 255) / 256 > 65535)
     return fail(TILEMIX_ERR_UNSUPPORTED,
                 "attn: hq, batch or query tiles per sequence above 65535");
   const int qbq = a->quant_block_q > 0 ? a->quant_block_q : 128;
@@ -257,17 +257,19 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   memset(&p, 0, sizeof(p));
   const CUtensorMapSwizzle i8sw =
       d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  // The kernel computes 128 x 64 score tiles; a 128-key routing tile is two
+  // compute tiles that read the same bit.
   bool maps = make_map(&p.tm_q, a->q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
                        a->hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_map(&p.tm_k, a->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
-                       a->hkv, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B) &&
+                       a->hkv, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_map(&p.tm_v, a->v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
-                       a->hkv, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B);
+                       a->hkv, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (maps && !fp16_only)
     maps = make_map(&p.tm_q8, a->q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
                     a->hq, d, 128, i8sw) &&
            make_map(&p.tm_k8, a->k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
-                    a->hkv, d, bn, i8sw);
+                    a->hkv, d, 64, i8sw);
   if (!maps) return fail(TILEMIX_ERR_CUDA, "attn: tensor map encoding failed");
 
   p.cu_seqlens = a->cu_seqlens;
@@ -286,9 +288,11 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   p.hkv = a->hkv;
   p.heads_per_kv = a->head_map ? 1 : a->hq / a->hkv;
   p.route_bm = a->block_m;
+  p.route_bn = bn;
   p.tm_route = (a->max_seqlen + a->block_m - 1) / a->block_m;
   p.tn_max = (a->max_seqlen + bn - 1) / bn;
   p.group = a->group;
+  p.tiles_per_bit = a->group * (bn / 64);
   p.quant_block_q = qbq;
   p.quant_block_k = qbk;
   p.nbq = (a->max_seqlen + qbq - 1) / qbq;
@@ -298,7 +302,7 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
       a->softmax_scale > 0.0f ? a->softmax_scale : 1.0f / std::sqrt(float(d));
   p.scale_log2 = scale * 1.4426950408889634f;
 
-  tilemix::AttnLaunchShape shape{d, bn, a->block_m == 64};
+  tilemix::AttnLaunchShape shape{d, a->block_m == 64};
   cudaError_t e = tilemix::launch_attn_prefill(p, shape, stream);
   if (e != cudaSuccess)
     return fail(TILEMIX_ERR_CUDA, "attn launch: %s", cudaGetErrorString(e));

@@ -176,14 +176,33 @@ def test_explicit_head_map(tm):
     compare(got["out"], ref)
 
 
-def test_int8_tiles_bitexact_dump(tm):
-    inp = small([700, 300], bm=128, bn=128, hkv=1, recipe="exact", cov=0.5)
+def _mask_past_route_row(dump, lens, bm, bn, fill=-1):
+    """Blank the keys past the last query of each routing row: every row of
+    the routing row masks them, and the kernel may skip them in 64-key
+    steps (the C ABI documents this)."""
+    out = dump.copy()
+    for b, L in enumerate(lens):
+        for m in range(out.shape[2]):
+            last = min((m + 1) * bm, int(L)) - 1
+            for n in range(out.shape[3]):
+                first_dead = max(0, last + 1 - n * bn)
+                if first_dead < bn:
+                    out[b, :, m, n, :, first_dead:] = fill
+    return out
+
+
+@pytest.mark.parametrize("bm,bn,g", [(128, 128, 1), (128, 64, 1), (64, 64, 2)])
+def test_int8_tiles_bitexact_dump(tm, bm, bn, g):
+    inp = small([700, 300], bm=bm, bn=bn, g=g, hkv=1, recipe="exact", cov=0.5)
     got = run_gpu(inp, want_dump=True)
     _, kw = run_oracle(inp, rows=np.array([0]))
     dump = oracle.qk_dump(inp["cu_seqlens"], 700, kw["q8"], kw["k8"],
-                          kw["mask"], hq=4, hkv=1, d=128, block_m=128,
-                          block_n=128, group=1, fill=-1)
-    assert np.array_equal(got["dump"], dump)
+                          kw["mask"], hq=4, hkv=1, d=128, block_m=bm,
+                          block_n=bn, group=g, fill=-1)
+    lens = inp["seqlens"]
+    assert np.array_equal(_mask_past_route_row(got["dump"], lens, bm, bn),
+                          _mask_past_route_row(dump, lens, bm, bn))
+    assert (_mask_past_route_row(dump, lens, bm, bn) != -1).any()
 
 
 def test_garbage_bits_in_illegal_groups_change_nothing(tm):
