@@ -34,9 +34,9 @@ cudaError_t launch_pack_mask(const uint8_t* route, const int32_t* cu_seqlens,
 struct AttnParams {
   CUtensorMap tm_q;   // fp16 Q  [T, hq, d], box {64, 128, 1}, 128B swizzle
   CUtensorMap tm_q8;  // int8 Q8 [T, hq, d], box {d, 128, 1}
-  CUtensorMap tm_k;   // fp16 K  [T, hkv, d], box {64, 64, 1}
-  CUtensorMap tm_k8;  // int8 K8 [T, hkv, d], box {d, 64, 1}
-  CUtensorMap tm_v;   // fp16 V  [T, hkv, d], box {64, 64, 1}
+  CUtensorMap tm_k;   // fp16 K  [T, hkv, d], box {64, 128, 1}
+  CUtensorMap tm_k8;  // int8 K8 [T, hkv, d], box {d, 128, 1}
+  CUtensorMap tm_v;   // fp16 V  [T, hkv, d], box {64, 128, 1}
   const int32_t* cu_seqlens;
   const int32_t* head_map;
   const uint64_t* mask;
@@ -53,7 +53,7 @@ struct AttnParams {
   int tm_route;      // ceil(max_seqlen / route_bm)
   int tn_max;        // ceil(max_seqlen / route_bn)
   int group;         // g: routing tiles per bit
-  int tiles_per_bit; // 64-key compute tiles per bit = g * route_bn / 64
+  int tiles_per_bit; // 64-key blocks per routing bit = g * route_bn / 64
   int quant_block_q, quant_block_k, nbq, nbk;
   int fp16_only;
   float scale_log2;  // softmax scale * log2(e)

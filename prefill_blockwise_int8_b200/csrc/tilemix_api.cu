@@ -257,19 +257,19 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   memset(&p, 0, sizeof(p));
   const CUtensorMapSwizzle i8sw =
       d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  // The kernel computes 128 x 64 score tiles; a 128-key routing tile is two
-  // compute tiles that read the same bit.
+  // The kernel computes 128 x 128 score tiles (a 64-key routing tile is one
+  // half of a compute tile).
   bool maps = make_map(&p.tm_q, a->q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
                        a->hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_map(&p.tm_k, a->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
-                       a->hkv, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
+                       a->hkv, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_map(&p.tm_v, a->v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
-                       a->hkv, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+                       a->hkv, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (maps && !fp16_only)
     maps = make_map(&p.tm_q8, a->q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
                     a->hq, d, 128, i8sw) &&
            make_map(&p.tm_k8, a->k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
-                    a->hkv, d, 64, i8sw);
+                    a->hkv, d, 128, i8sw);
   if (!maps) return fail(TILEMIX_ERR_CUDA, "attn: tensor map encoding failed");
 
   p.cu_seqlens = a->cu_seqlens;
