@@ -71,7 +71,7 @@ struct Cfg {
   static constexpr int kK8Off = align1k(kK16Bytes);
   static constexpr int kKSlotBytes = align1k(kK8Off + kK8Bytes);
   static constexpr int kVSlotBytes = align1k(kVBytes);
-  static constexpr int kRedBytes = DUAL ? 4096 : 0;  // row max / sum exchange
+  static constexpr int kRedBytes = 2048;  // row max / sum exchange [2][2][128]
   static constexpr int kBarBytes = 512;
   static constexpr int kAvail =
       kSmemBudget - 1024 - kBarBytes - kRedBytes - kRing0;
@@ -95,6 +95,9 @@ struct Cfg {
   // tiles; in spare columns with one, where the two warpgroups read the
   // fp16 S region while the other may already store P.
   static constexpr int kP = DUAL ? 3 * kBN : 0;
+  // P of warpgroup wg's 64 keys (32 columns): over the S columns it read
+  // with two query tiles; in the spare columns with one.
+  static constexpr int p_col(int wg) { return DUAL ? kP + 32 * wg : kHalf * wg; }
   static constexpr int kTileCols = DUAL ? 512 : 256;
   static constexpr int kTmemCols = 512;
   static_assert(kOCol + D <= kTileCols, "TMEM overflow");
@@ -107,7 +110,7 @@ struct Cfg {
   static constexpr int kBarS = kBarVEmpty + kVStages;  // [tile]
   static constexpr int kBarP = kBarS + 2;              // [tile]
   static constexpr int kBarO = kBarP + 2;              // [tile]
-  static constexpr int kBarRed = kBarO + 2;            // one tile: [2]
+  static constexpr int kBarRed = kBarO + 2;            // [parity]
   static constexpr int kBarDrain = kBarRed + 2;
   static constexpr int kNumBars = kBarDrain + 1;
   static_assert(kNumBars * 8 + 16 <= kBarBytes, "barrier area");
@@ -132,6 +135,83 @@ __device__ __forceinline__ uint64_t desc_k_i8(uint32_t base, int ks) {
 // ks = K-step of 16 keys.  LBO = chunk stride, SBO = 8 keys.
 __device__ __forceinline__ uint64_t desc_v(uint32_t base, int ks) {
   return smem_desc(base + ks * 16 * 128, kBN * 128, 1024, kSwizzle128);
+}
+
+// Row max of 64 scores held as raw bits (INT32 accumulators when I8, fp32
+// otherwise).  With MASKED, columns j > hl are left out.  The masked /
+// unmasked choice is made once per 64-key half, not per element.
+template <bool I8, bool MASKED>
+__device__ __forceinline__ float max64(const uint32_t (&sv)[64], int hl) {
+  if (I8) {
+    int a0 = INT_MIN, a1 = INT_MIN, a2 = INT_MIN, a3 = INT_MIN;
+#pragma unroll
+    for (int j = 0; j < 64; j += 4) {
+      a0 = max(a0, (!MASKED || j <= hl) ? static_cast<int>(sv[j]) : INT_MIN);
+      a1 = max(a1, (!MASKED || j + 1 <= hl) ? static_cast<int>(sv[j + 1]) : INT_MIN);
+      a2 = max(a2, (!MASKED || j + 2 <= hl) ? static_cast<int>(sv[j + 2]) : INT_MIN);
+      a3 = max(a3, (!MASKED || j + 3 <= hl) ? static_cast<int>(sv[j + 3]) : INT_MIN);
+    }
+    if (MASKED && hl < 0) return -CUDART_INF_F;
+    return static_cast<float>(max(max(a0, a1), max(a2, a3)));
+  } else {
+    auto g = [&](int j) {
+      return (!MASKED || j <= hl) ? __uint_as_float(sv[j]) : -CUDART_INF_F;
+    };
+    float a0 = -CUDART_INF_F, a1 = -CUDART_INF_F, a2 = -CUDART_INF_F,
+          a3 = -CUDART_INF_F;
+#pragma unroll
+    for (int j = 0; j < 64; j += 8) {
+      a0 = fmax3(a0, g(j), g(j + 1));
+      a1 = fmax3(a1, g(j + 2), g(j + 3));
+      a2 = fmax3(a2, g(j + 4), g(j + 5));
+      a3 = fmax3(a3, g(j + 6), g(j + 7));
+    }
+    return fmax3(a0, a1, fmaxf(a2, a3));
+  }
+}
+
+// P = 2^(S c - m) of 32 scores as 16 packed fp16 pairs (key 2i in the low
+// half of pk[i]), added to four packed partial sums.  INT32 accumulators
+// convert to fp32 exactly (|acc| <= 127^2 d < 2^22) by the bias trick, on
+// the integer and FMA pipes rather than the conversion unit.  With MASKED,
+// columns j > hl give exactly 0.  With TRACK, xmax accumulates the largest
+// exponent S c - m over the legal columns.
+template <bool I8, bool MASKED, bool TRACK>
+__device__ __forceinline__ void exp32(const uint32_t (&sv)[32], float c,
+                                      float m, int hl, uint32_t* pk,
+                                      float2& ps0, float2& ps1, float2& ps2,
+                                      float2& ps3, float& xmax) {
+  const float2 c2 = make_float2(c, c);
+  const float2 nm2 = make_float2(-m, -m);
+  float xa = -CUDART_INF_F, xb = -CUDART_INF_F;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int j = 2 * i;
+    float2 sc = make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
+    if (I8) {
+      sc = __fadd2_rn(make_float2(__uint_as_float(sv[j] + kIntBiasBits),
+                                  __uint_as_float(sv[j + 1] + kIntBiasBits)),
+                      make_float2(-kIntBias, -kIntBias));
+    }
+    float2 x = __ffma2_rn(sc, c2, nm2);
+    if (MASKED) {  // 2^-inf = 0, also when c == 0
+      x.x = (j <= hl) ? x.x : -CUDART_INF_F;
+      x.y = (j + 1 <= hl) ? x.y : -CUDART_INF_F;
+    }
+    if (TRACK) {
+      if (i & 1) xb = fmax3(xb, x.x, x.y);
+      else xa = fmax3(xa, x.x, x.y);
+    }
+    const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    switch (i & 3) {
+      case 0: ps0 = __fadd2_rn(ps0, pr); break;
+      case 1: ps1 = __fadd2_rn(ps1, pr); break;
+      case 2: ps2 = __fadd2_rn(ps2, pr); break;
+      default: ps3 = __fadd2_rn(ps3, pr); break;
+    }
+    pk[i] = pack_half2(pr.x, pr.y);
+  }
+  if (TRACK) xmax = fmax3(xmax, xa, xb);
 }
 
 // Routing state of one 128-row query tile.
@@ -221,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto sQ8 = [&](int t) { return smem + C::kQ8Off + t * C::kQ8Bytes; };
   auto kslot = [&](int s) { return smem + C::kRing0 + s * C::kKSlotBytes; };
   auto vslot = [&](int s) { return smem + C::kVRing0 + s * C::kVSlotBytes; };
-  // one query tile: [max | sum][tile parity][warpgroup][row]
+  // row max / sum exchange between the softmax warpgroups: [slot][wg][row]
   float* red = reinterpret_cast<float*>(smem + C::kRedOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
@@ -239,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars[C::kBarS + i], 1);
-      mbar_init(&bars[C::kBarP + i], DUAL ? 256 : 128);
+      mbar_init(&bars[C::kBarP + i], 256);
       mbar_init(&bars[C::kBarO + i], 1);
       mbar_init(&bars[C::kBarRed + i], 256);
     }
@@ -406,8 +486,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tb = tmem + t * C::kTileCols;
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks)
-          mma_f16_ts(tb + C::kOCol, tb + C::kP + ks * 8, desc_v(vb, ks),
-                     idesc_pv, (n > 0 || ks > 0) ? 1u : 0u);
+          mma_f16_ts(tb + C::kOCol, tb + C::p_col(ks >> 2) + (ks & 3) * 8,
+                     desc_v(vb, ks), idesc_pv, (n > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&bars[C::kBarO + t]);
         return true;
       };
@@ -436,51 +516,59 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // =================== softmax warps 0-7 ===================
-    // Two query tiles: warpgroup wg serves tile wg, all 128 keys of a tile.
-    // One query tile (DUAL): warpgroup wg serves keys 64*wg .. 64*wg+63.
+    // Warpgroup wg takes keys 64*wg .. 64*wg+63 of every row (thread = row =
+    // TMEM lane) of each query tile.  Both warpgroups work on the CTA's
+    // query tiles one after the other (tile 0 then tile 1 for each key
+    // tile), so that one tile's softmax overlaps the other tile's P V and
+    // Q K^T on the tensor cores.  The row max is combined through shared
+    // memory every tile; each warpgroup keeps the sum of its own keys and
+    // the two are added once, at the end.
     const int wg = warp >> 2;
-    const int t = DUAL ? 0 : wg;
-    const int r = threadIdx.x & 127;  // score row = TMEM lane
-    constexpr int kCols = DUAL ? kHalf : kBN;  // score columns per thread
-    const int c0 = DUAL ? wg * kHalf : 0;      // first column of this thread
-    const TileRoute R = rt(t);
-    if (R.n_last >= 0) {
-      const int r_local = row_base + t * kBM + r;
-      const bool valid = r_local < len;
-      const int rh = DUAL ? (r >> 6) : 0;  // routing row half
-      const uint64_t my_w = rh ? R.w1 : R.w0;
-      const int my_nl = rh ? R.nl1 : R.nl0;
-      const uint32_t tb = tmem + t * C::kTileCols;
-      const uint32_t lane_addr =
-          tb + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-      const int key_lim = min(r_local, len - 1);  // keys j <= key_lim legal
-      float sq = 0.0f;
-      if (routed)
-        sq = p.q_scale[(static_cast<size_t>(h) * p.batch + b) * p.nbq +
-                       key_lim / p.quant_block_q];
-      const float* kscale =
-          routed ? p.k_scale + (static_cast<size_t>(hk) * p.batch + b) * p.nbk
-                 : nullptr;
-      // K scales of the next tile are fetched while this one is processed.
-      auto ksc = [&](int n, int kh) {
-        const int blk = (n * kBN + kh * kHalf) / p.quant_block_k;
-        return kscale[min(blk, p.nbk - 1)];
-      };
-      float sk0_next = 0.f, sk1_next = 0.f;
-      if (routed) {
-        sk0_next = ksc(0, 0);
-        sk1_next = ksc(0, 1);
-      }
+    const int r = threadIdx.x & 127;
+    const int c0 = wg * kHalf;  // first key of this thread inside a key tile
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float* kscale =
+        routed ? p.k_scale + (static_cast<size_t>(hk) * p.batch + b) * p.nbk
+               : nullptr;
+    // K scale of this thread's 64 keys; the next key tile's is fetched while
+    // the current one is processed.
+    auto ksc = [&](int n) {
+      const int blk = (n * kBN + c0) / p.quant_block_k;
+      return kscale[min(blk, p.nbk - 1)];
+    };
+    float sk_next = routed ? ksc(0) : 0.0f;
+    // running max and (this warpgroup's) sum of each query tile's rows
+    float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.0f, l1 = 0.0f;
+    uint32_t u = 0;  // tiles processed so far: parity of the exchange slot
+    bool ok = true;
+    // Combine a per-row value with the other warpgroup's (max or sum).
+    auto exchange = [&](float v, bool& good) -> float {
+      float* slot = red + (u & 1) * 256;
+      slot[wg * 128 + r] = v;
+      mbar_arrive(&bars[C::kBarRed + (u & 1)]);
+      const bool got = mbar_wait(&bars[C::kBarRed + (u & 1)], (u >> 1) & 1,
+                                 abort_flag);
+      good = __all_sync(0xffffffffu, got);
+      const float other = slot[(1 - wg) * 128 + r];
+      ++u;
+      return other;
+    };
 
-      float m_run = -CUDART_INF_F;
-      float l_run = 0.0f;
-      bool ok = true;
-      for (int n = 0; n <= R.n_last; ++n) {
-        const float sk0 = sk0_next, sk1 = sk1_next;
-        if (routed && n < R.n_last) {
-          sk0_next = ksc(n + 1, 0);
-          sk1_next = ksc(n + 1, 1);
-        }
+    for (int n = 0; n <= n_end && ok; ++n) {
+      const float sk = sk_next;
+      if (routed && n < n_end) sk_next = ksc(n + 1);
+#pragma unroll 1
+      for (int t = 0; t < kQT; ++t) {
+        const TileRoute& R = rt(t);
+        if (n > R.n_last) continue;  // same decision in both warpgroups
+        const int r_local = row_base + t * kBM + r;
+        const int rh = DUAL ? (r >> 6) : 0;  // routing row half
+        const uint64_t my_w = rh ? R.w1 : R.w0;
+        const int my_nl = rh ? R.nl1 : R.nl0;
+        const int key_lim = min(r_local, len - 1);  // keys j <= key_lim legal
+        const uint32_t tb = tmem + t * C::kTileCols;
+        const uint32_t lane_addr = tb + lane_off;
+
         // Exits stay warp-uniform: the tcgen05.ld/st below are .sync.aligned.
         const bool got_s = mbar_wait(&bars[C::kBarS + t], n & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got_s)) {
@@ -488,237 +576,167 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        // Path of each 64-key half of this thread's columns for this row
-        // (its routing row half).  kLH local halves, global half c0/64 + hh.
-        constexpr int kLH = kCols / kHalf;
-        bool i8l[kLH];
-        float csl[kLH];
+        // Path of this thread's 64 keys for its routing row half.  Keys past
+        // every row of the tile: the MMA wrote the first half's path there
+        // (values masked below either way).
+        const int n64 = 2 * n + wg;
+        const int nb = (!DUAL && n64 > my_nl) ? 2 * n : n64;
+        const bool i8 =
+            (nb <= my_nl) && (((my_w >> (nb / tpb)) & 1ull) != 0);
+        float c = p.scale_log2;
+        if (i8)
+          c *= sk * p.q_scale[(static_cast<size_t>(h) * p.batch + b) * p.nbq +
+                              key_lim / p.quant_block_q];
+        uint32_t sv[kHalf];
+        const uint32_t scol = lane_addr + (i8 ? C::kS8 : C::kS16) + c0;
+        tmem_ld32(scol, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld_wait();
+        if (p.qk_dump && r_local < len && i8 && n64 <= my_nl) {
+          const int rrow = r_local / p.route_bm;
+          const int rr = r_local - rrow * p.route_bm;
+          const int key0 = n64 * kHalf;
+          const int nr = key0 / p.route_bn;
+          int32_t* dst =
+              p.qk_dump +
+              ((((static_cast<size_t>(b) * p.hq + h) * p.tm_route + rrow) *
+                    p.tn_max +
+                nr) *
+                   p.route_bm +
+               rr) *
+                  p.route_bn +
+              (key0 - nr * p.route_bn);
+          const int keys_left = len - key0;  // keys inside the sequence
 #pragma unroll
-        for (int hh = 0; hh < kLH; ++hh) {
-          const int n64 = 2 * n + c0 / kHalf + hh;
-          i8l[hh] = (n64 <= my_nl) && (((my_w >> (n64 / tpb)) & 1ull) != 0);
+          for (int j = 0; j < kHalf; ++j)
+            if (j < keys_left) dst[j] = static_cast<int32_t>(sv[j]);
         }
-        // Keys past every row of the tile: the MMA wrote the other half's
-        // path there; those values are masked below either way.
-        if (!DUAL && 2 * n + 1 > my_nl) i8l[kLH - 1] = i8l[0];
-#pragma unroll
-        for (int hh = 0; hh < kLH; ++hh)
-          csl[hh] = i8l[hh] ? p.scale_log2 * sq *
-                                  ((c0 / kHalf + hh) ? sk1 : sk0)
-                            : p.scale_log2;
-        const int lim = key_lim - n * kBN - c0;  // columns j <= lim are legal
-        const bool full = lim >= kCols - 1;
-        auto s_col = [&](int hh) {
-          return lane_addr + (i8l[hh] ? C::kS8 : C::kS16) + c0 + hh * kHalf;
-        };
-
-        // Pass 1: row max, 64 columns at a time (the scores stay in TMEM).
-        // INT8 halves take the integer max of the raw accumulators.
-        float m_tile = -CUDART_INF_F;
-#pragma unroll
-        for (int hh = 0; hh < kLH; ++hh) {
-          uint32_t sv[kHalf];
-          tmem_ld32(s_col(hh), *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-          tmem_ld32(s_col(hh) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-          tmem_ld_wait();
-          const int hl = lim - hh * kHalf;  // legal columns of this half: <= hl
-          if (p.qk_dump && valid && i8l[hh] && 2 * n + c0 / kHalf + hh <= my_nl) {
-            const int n64 = 2 * n + c0 / kHalf + hh;
-            const int rrow = r_local / p.route_bm;
-            const int rr = r_local - rrow * p.route_bm;
-            const int key0 = n64 * kHalf;
-            const int nr = key0 / p.route_bn;
-            int32_t* dst =
-                p.qk_dump +
-                ((((static_cast<size_t>(b) * p.hq + h) * p.tm_route + rrow) *
-                      p.tn_max +
-                  nr) *
-                     p.route_bm +
-                 rr) *
-                    p.route_bn +
-                (key0 - nr * p.route_bn);
-            const int keys_left = len - key0;  // keys inside the sequence
-#pragma unroll
-            for (int j = 0; j < kHalf; ++j)
-              if (j < keys_left) dst[j] = static_cast<int32_t>(sv[j]);
-          }
-          float mx;
-          if (i8l[hh]) {
-            int a0 = INT_MIN, a1 = INT_MIN, a2 = INT_MIN, a3 = INT_MIN;
-#pragma unroll
-            for (int j = 0; j < kHalf; j += 4) {
-              const bool fullh = hl >= kHalf - 1;
-              a0 = max(a0, (fullh || j <= hl) ? static_cast<int>(sv[j]) : INT_MIN);
-              a1 = max(a1, (fullh || j + 1 <= hl) ? static_cast<int>(sv[j + 1]) : INT_MIN);
-              a2 = max(a2, (fullh || j + 2 <= hl) ? static_cast<int>(sv[j + 2]) : INT_MIN);
-              a3 = max(a3, (fullh || j + 3 <= hl) ? static_cast<int>(sv[j + 3]) : INT_MIN);
-            }
-            const int im = max(max(a0, a1), max(a2, a3));
-            mx = (hl < 0) ? -CUDART_INF_F : static_cast<float>(im);
-          } else {
-            float a0 = -CUDART_INF_F, a1 = -CUDART_INF_F, a2 = -CUDART_INF_F,
-                  a3 = -CUDART_INF_F;
-            auto g = [&](int j) {
-              return (hl >= kHalf - 1 || j <= hl) ? __uint_as_float(sv[j])
-                                                  : -CUDART_INF_F;
-            };
-#pragma unroll
-            for (int j = 0; j < kHalf; j += 8) {
-              a0 = fmax3(a0, g(j), g(j + 1));
-              a1 = fmax3(a1, g(j + 2), g(j + 3));
-              a2 = fmax3(a2, g(j + 4), g(j + 5));
-              a3 = fmax3(a3, g(j + 6), g(j + 7));
-            }
-            mx = fmax3(a0, a1, fmaxf(a2, a3));
-          }
-          if (mx != -CUDART_INF_F) m_tile = fmaxf(m_tile, mx * csl[hh]);
+        const int hl = key_lim - n * kBN - c0;  // legal columns: j <= hl
+        const bool fullh = hl >= kHalf - 1;
+        const float mx = i8 ? (fullh ? max64<true, false>(sv, hl)
+                                     : max64<true, true>(sv, hl))
+                            : (fullh ? max64<false, false>(sv, hl)
+                                     : max64<false, true>(sv, hl));
+        const float m_half = (mx == -CUDART_INF_F) ? -CUDART_INF_F : mx * c;
+        bool good = true;
+        const float m_tile = fmaxf(m_half, exchange(m_half, good));
+        if (!good) {
+          ok = false;
+          break;
         }
-        if (DUAL) {
-          // the two warpgroups hold the two halves of each row
-          red[(n & 1) * 256 + wg * 128 + r] = m_tile;
-          mbar_arrive(&bars[C::kBarRed + (n & 1)]);
-          const bool got_r =
-              mbar_wait(&bars[C::kBarRed + (n & 1)], (n >> 1) & 1, abort_flag);
-          if (!__all_sync(0xffffffffu, got_r)) {
-            ok = false;
-            break;
-          }
-          m_tile = fmaxf(m_tile, red[(n & 1) * 256 + (1 - wg) * 128 + r]);
-        }
+        float m_run = t ? m1 : m0;
+        float l_run = t ? l1 : l0;
         const float m_new = fmaxf(m_run, m_tile);
         const bool need = m_new > m_run + kRescaleThreshold;
-
-        if (n > 0) {
-          // O holds P V of every tile before n once PV(n-1) completed.
-          const bool got_o =
-              mbar_wait(&bars[C::kBarO + t], (n - 1) & 1, abort_flag);
-          if (!__all_sync(0xffffffffu, got_o)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, need)) {
-            const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
-            // with one query tile each warpgroup rescales half of O
-            constexpr int kOCols = DUAL ? D / 2 : D;
-            const int o0 = DUAL ? wg * (D / 2) : 0;
-#pragma unroll
-            for (int oc = 0; oc < kOCols; oc += 32) {
-              uint32_t o[32];
-              tmem_ld32(lane_addr + C::kOCol + o0 + oc, o);
-              tmem_ld_wait();
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-              tmem_st32(lane_addr + C::kOCol + o0 + oc, o);
-            }
-          }
-        }
+        const float m_old = m_run;
         if (need) {
           l_run *= ex2_approx(m_run - m_new);
           m_run = m_new;
         }
-        // Pass 2: P = 2^(x - m) as fp16 pairs, key 2i of this thread's
-        // columns in the low half of P column (c0 / 2 + i); packed partial
-        // sums.  INT32 accumulators convert to fp32 exactly (|acc| <= 127^2 d
-        // < 2^22) on the integer and FMA pipes, not the conversion unit.
+        // P = 2^(S c - m) of this thread's 64 keys as fp16 pairs over the S
+        // columns it has just read (key 2i in the low half of column i).
         float2 ps0 = make_float2(0.f, 0.f), ps1 = ps0, ps2 = ps0, ps3 = ps0;
-        const float2 nm2 = make_float2(-m_run, -m_run);
+        float unused_max = 0.0f;
 #pragma unroll
-        for (int hh = 0; hh < kLH; ++hh) {
-          uint32_t sv[kHalf];
-          tmem_ld32(s_col(hh), *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-          tmem_ld32(s_col(hh) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-          tmem_ld_wait();
-          if (i8l[hh]) {
-#pragma unroll
-            for (int j = 0; j < kHalf; j += 2) {
-              const float2 biased =
-                  make_float2(__uint_as_float(sv[j] + kIntBiasBits),
-                              __uint_as_float(sv[j + 1] + kIntBiasBits));
-              const float2 v =
-                  __fadd2_rn(biased, make_float2(-kIntBias, -kIntBias));
-              sv[j] = __float_as_uint(v.x);
-              sv[j + 1] = __float_as_uint(v.y);
-            }
+        for (int q = 0; q < 2; ++q) {
+          uint32_t pk[16];
+          const int hq = hl - 32 * q;
+          const uint32_t(&sq32)[32] =
+              *reinterpret_cast<const uint32_t(*)[32]>(&sv[32 * q]);
+          uint32_t* pkq = pk;
+          const bool fullq = hq >= 31;
+          if (i8) {
+            if (fullq) exp32<true, false, false>(sq32, c, m_run, hq, pkq, ps0, ps1, ps2, ps3, unused_max);
+            else exp32<true, true, false>(sq32, c, m_run, hq, pkq, ps0, ps1, ps2, ps3, unused_max);
+          } else {
+            if (fullq) exp32<false, false, false>(sq32, c, m_run, hq, pkq, ps0, ps1, ps2, ps3, unused_max);
+            else exp32<false, true, false>(sq32, c, m_run, hq, pkq, ps0, ps1, ps2, ps3, unused_max);
           }
-          const float2 c2 = make_float2(csl[hh], csl[hh]);
-          const int hl = lim - hh * kHalf;
-          uint32_t pk[32];
+          tmem_st16(lane_addr + C::p_col(wg) + 16 * q, pk);
+        }
+        if (n > 0 && __any_sync(0xffffffffu, need)) {
+          // S_t(n) is ready, so P V_t(n-1) completed (the MMA thread issues
+          // Q K^T_t(n) after it): O_t can be rescaled now.  Each warpgroup
+          // rescales half of O's columns.
+          const float alpha = need ? ex2_approx(m_old - m_new) : 1.0f;
+          const int o0 = wg * (D / 2);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int j = 2 * i;
-            const float2 x = __ffma2_rn(
-                make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])),
-                c2, nm2);
-            float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            if (!full) {  // masked keys: exactly 0
-              pr.x = (j <= hl) ? pr.x : 0.0f;
-              pr.y = (j + 1 <= hl) ? pr.y : 0.0f;
-            }
-            switch (i & 3) {
-              case 0: ps0 = __fadd2_rn(ps0, pr); break;
-              case 1: ps1 = __fadd2_rn(ps1, pr); break;
-              case 2: ps2 = __fadd2_rn(ps2, pr); break;
-              default: ps3 = __fadd2_rn(ps3, pr); break;
-            }
-            pk[i] = pack_half2(pr.x, pr.y);
+          for (int oc = 0; oc < D / 2; oc += 32) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + C::kOCol + o0 + oc, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            tmem_st32(lane_addr + C::kOCol + o0 + oc, o);
           }
-          tmem_st32(lane_addr + C::kP + (c0 + hh * kHalf) / 2, pk);
         }
         const float2 s4 = __fadd2_rn(__fadd2_rn(ps0, ps1), __fadd2_rn(ps2, ps3));
-        float lsum = s4.x + s4.y;
-        if (DUAL) red[512 + (n & 1) * 256 + wg * 128 + r] = lsum;
+        l_run += s4.x + s4.y;
+        if (t) {
+          m1 = m_run;
+          l1 = l_run;
+        } else {
+          m0 = m_run;
+          l0 = l_run;
+        }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars[C::kBarP + t]);
-        if (DUAL) {
-          // both halves' sums are in shared memory once the P barrier
-          // (both warpgroups' arrivals) completes
-          const bool got_p = mbar_wait(&bars[C::kBarP + t], n & 1, abort_flag);
-          if (!__all_sync(0xffffffffu, got_p)) {
-            ok = false;
-            break;
-          }
-          lsum += red[512 + (n & 1) * 256 + (1 - wg) * 128 + r];
-        }
-        l_run += lsum;
-      }
-
-      const bool got_last =
-          ok && mbar_wait(&bars[C::kBarO + t], R.n_last & 1, abort_flag);
-      if (__all_sync(0xffffffffu, got_last)) {
-        tc_fence_after();
-        const float inv_l = 1.0f / l_run;
-        constexpr int kOCols = DUAL ? D / 2 : D;
-        const int o0 = DUAL ? wg * (D / 2) : 0;
-        uint16_t* orow =
-            p.out + (static_cast<size_t>(start + r_local) * p.hq + h) * D + o0;
-#pragma unroll
-        for (int oc = 0; oc < kOCols; oc += 32) {
-          uint32_t o[32];
-          tmem_ld32(lane_addr + C::kOCol + o0 + oc, o);
-          tmem_ld_wait();
-          uint32_t hv[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            hv[j] = pack_half2(__uint_as_float(o[2 * j]) * inv_l,
-                               __uint_as_float(o[2 * j + 1]) * inv_l);
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + oc);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(hv[4 * v], hv[4 * v + 1], hv[4 * v + 2],
-                                  hv[4 * v + 3]);
-          }
-        }
-        if (p.lse && valid && wg == t)
-          p.lse[static_cast<size_t>(h) * p.total_tokens + start + r_local] =
-              (m_run + __log2f(l_run)) * 0.69314718055994530942f;
-      } else {
-        fail();
       }
     }
+
+    // Epilogue of each query tile: O / l, both warpgroups' sums combined;
+    // each warpgroup stores half of O's columns.
+#pragma unroll 1
+    for (int t = 0; t < kQT; ++t) {
+      const TileRoute& R = rt(t);
+      if (R.n_last < 0) continue;
+      const bool got_last =
+          ok && mbar_wait(&bars[C::kBarO + t], R.n_last & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got_last)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      bool good = true;
+      const float l_mine = t ? l1 : l0;
+      const float l_run = l_mine + exchange(l_mine, good);
+      if (!good) {
+        ok = false;
+        break;
+      }
+      const float m_run = t ? m1 : m0;
+      const int r_local = row_base + t * kBM + r;
+      const bool valid = r_local < len;
+      const uint32_t lane_addr = tmem + t * C::kTileCols + lane_off;
+      const float inv_l = 1.0f / l_run;
+      const int o0 = wg * (D / 2);
+      uint16_t* orow =
+          p.out + (static_cast<size_t>(start + r_local) * p.hq + h) * D + o0;
+#pragma unroll
+      for (int oc = 0; oc < D / 2; oc += 32) {
+        uint32_t o[32];
+        tmem_ld32(lane_addr + C::kOCol + o0 + oc, o);
+        tmem_ld_wait();
+        uint32_t hv[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          hv[j] = pack_half2(__uint_as_float(o[2 * j]) * inv_l,
+                             __uint_as_float(o[2 * j + 1]) * inv_l);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + oc);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(hv[4 * v], hv[4 * v + 1], hv[4 * v + 2],
+                                hv[4 * v + 3]);
+        }
+      }
+      if (p.lse && valid && wg == 0)
+        p.lse[static_cast<size_t>(h) * p.total_tokens + start + r_local] =
+            (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+    }
+    if (!ok) fail();
   }
 
   tc_fence_before();
