@@ -142,31 +142,37 @@ __device__ __forceinline__ uint64_t desc_v(uint32_t base, int ks) {
 // unmasked choice is made once per 64-key half, not per element.
 template <bool I8, bool MASKED>
 __device__ __forceinline__ float max64(const uint32_t (&sv)[64], int hl) {
+  // eight independent 3-input chains of depth four, then a short tree
   if (I8) {
-    int a0 = INT_MIN, a1 = INT_MIN, a2 = INT_MIN, a3 = INT_MIN;
+    auto g = [&](int j) {
+      return (!MASKED || j <= hl) ? static_cast<int>(sv[j]) : INT_MIN;
+    };
+    int a[8];
 #pragma unroll
-    for (int j = 0; j < 64; j += 4) {
-      a0 = max(a0, (!MASKED || j <= hl) ? static_cast<int>(sv[j]) : INT_MIN);
-      a1 = max(a1, (!MASKED || j + 1 <= hl) ? static_cast<int>(sv[j + 1]) : INT_MIN);
-      a2 = max(a2, (!MASKED || j + 2 <= hl) ? static_cast<int>(sv[j + 2]) : INT_MIN);
-      a3 = max(a3, (!MASKED || j + 3 <= hl) ? static_cast<int>(sv[j + 3]) : INT_MIN);
-    }
+    for (int k = 0; k < 8; ++k) a[k] = max(g(2 * k), g(2 * k + 1));
+#pragma unroll
+    for (int j = 16; j < 64; j += 16)
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        a[k] = __vimax3_s32(a[k], g(j + 2 * k), g(j + 2 * k + 1));
+    const int m = __vimax3_s32(__vimax3_s32(a[0], a[1], a[2]),
+                               __vimax3_s32(a[3], a[4], a[5]), max(a[6], a[7]));
     if (MASKED && hl < 0) return -CUDART_INF_F;
-    return static_cast<float>(max(max(a0, a1), max(a2, a3)));
+    return static_cast<float>(m);
   } else {
     auto g = [&](int j) {
       return (!MASKED || j <= hl) ? __uint_as_float(sv[j]) : -CUDART_INF_F;
     };
-    float a0 = -CUDART_INF_F, a1 = -CUDART_INF_F, a2 = -CUDART_INF_F,
-          a3 = -CUDART_INF_F;
+    float a[8];
 #pragma unroll
-    for (int j = 0; j < 64; j += 8) {
-      a0 = fmax3(a0, g(j), g(j + 1));
-      a1 = fmax3(a1, g(j + 2), g(j + 3));
-      a2 = fmax3(a2, g(j + 4), g(j + 5));
-      a3 = fmax3(a3, g(j + 6), g(j + 7));
-    }
-    return fmax3(a0, a1, fmaxf(a2, a3));
+    for (int k = 0; k < 8; ++k) a[k] = fmaxf(g(2 * k), g(2 * k + 1));
+#pragma unroll
+    for (int j = 16; j < 64; j += 16)
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        a[k] = fmax3(a[k], g(j + 2 * k), g(j + 2 * k + 1));
+    return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]),
+                 fmaxf(a[6], a[7]));
   }
 }
 
@@ -319,9 +325,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars[C::kBarS + i], 1);
-      mbar_init(&bars[C::kBarP + i], 256);
+      mbar_init(&bars[C::kBarP + i], 8);   // one arrival per softmax warp
       mbar_init(&bars[C::kBarO + i], 1);
-      mbar_init(&bars[C::kBarRed + i], 256);
+      mbar_init(&bars[C::kBarRed + i], 8);
     }
     mbar_init(&bars[C::kBarDrain], 1);
     *abort_flag = 0;
@@ -537,6 +543,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       return kscale[min(blk, p.nbk - 1)];
     };
     float sk_next = routed ? ksc(0) : 0.0f;
+    // softmax scale (log2 units) times the Q block scale of this thread's row
+    // in each query tile: the INT8 path's S c = (Q8 K8^T) sq sk scale log2(e)
+    auto qsc = [&](int t) {
+      const int key_lim = min(row_base + t * kBM + r, len - 1);
+      return (routed && key_lim >= 0)
+                 ? p.scale_log2 *
+                       p.q_scale[(static_cast<size_t>(h) * p.batch + b) * p.nbq +
+                                 key_lim / p.quant_block_q]
+                 : 0.0f;
+    };
+    const float cq0 = qsc(0), cq1 = kQT > 1 ? qsc(1) : 0.0f;
     // running max and (this warpgroup's) sum of each query tile's rows
     float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.0f, l1 = 0.0f;
     uint32_t u = 0;  // tiles processed so far: parity of the exchange slot
@@ -545,7 +562,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto exchange = [&](float v, bool& good) -> float {
       float* slot = red + (u & 1) * 256;
       slot[wg * 128 + r] = v;
-      mbar_arrive(&bars[C::kBarRed + (u & 1)]);
+      __syncwarp();  // orders the lanes' stores before lane 0's release
+      if (lane == 0) mbar_arrive(&bars[C::kBarRed + (u & 1)]);
       const bool got = mbar_wait(&bars[C::kBarRed + (u & 1)], (u >> 1) & 1,
                                  abort_flag);
       good = __all_sync(0xffffffffu, got);
@@ -583,10 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nb = (!DUAL && n64 > my_nl) ? 2 * n : n64;
         const bool i8 =
             (nb <= my_nl) && (((my_w >> (nb / tpb)) & 1ull) != 0);
-        float c = p.scale_log2;
-        if (i8)
-          c *= sk * p.q_scale[(static_cast<size_t>(h) * p.batch + b) * p.nbq +
-                              key_lim / p.quant_block_q];
+        const float c = i8 ? (t ? cq1 : cq0) * sk : p.scale_log2;
         uint32_t sv[kHalf];
         const uint32_t scol = lane_addr + (i8 ? C::kS8 : C::kS16) + c0;
         tmem_ld32(scol, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
@@ -682,7 +697,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bars[C::kBarP + t]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[C::kBarP + t]);
       }
     }
 
