@@ -10,7 +10,8 @@
 // HBM-bound: one CTA reads one block (up to 32 KB of fp16) once into
 // registers with 16-byte loads, reduces the absmax, and writes the codes
 // with 8-byte stores.  Rows of a block are strided by heads * d in memory,
-// each row contiguous.
+// each row contiguous.  The per-element IEEE division is replaced by a
+// multiply with the reciprocal wherever that provably gives the same code.
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -20,14 +21,35 @@ namespace tilemix {
 namespace {
 
 constexpr int kQThreads = 256;
-constexpr int kMaxVecs = 16;  // 16-byte vectors per thread: block*d <= 32768
 
+// code = rint(fl(x / s)) without a division per element: y = x * fl(1/s)
+// lies within a few ulp of fl(x / s) (|y| <= 128, so within 2^-15), hence
+// both round to the same integer unless y is within that distance of a
+// half-integer; those rare elements take the IEEE division.
+__device__ __forceinline__ int quant_code(float x, float s, float r) {
+  const float y = x * r;
+  const float t = rintf(y);
+  const float frac = fabsf(y - t);  // in [0, 0.5] (+ rounding)
+  int q;
+  if (frac < 0.5f - 0x1p-13f) {
+    q = static_cast<int>(t);
+  } else {
+    q = __float2int_rn(__fdiv_rn(x, s));
+  }
+  return max(-127, min(127, q));
+}
+
+// VPT 16-byte vectors (8 halves) per thread; VPR vectors per row (d / 8),
+// 0 = taken from vpr_rt at run time.
+template <int VPT, int VPR>
 __global__ void __launch_bounds__(kQThreads)
     quantize_kernel(const __half* __restrict__ x,
                     const int32_t* __restrict__ cu_seqlens, int batch,
-                    int max_seqlen, int total_tokens, int heads, int d,
-                    int block, int nblk, int8_t* __restrict__ x8,
+                    int max_seqlen, int total_tokens, int heads, int block,
+                    int nblk, int vpr_rt, int8_t* __restrict__ x8,
                     float* __restrict__ scale, int32_t* status) {
+  const int vpr = VPR > 0 ? VPR : vpr_rt;
+  const int d = vpr * 8;
   const int t = blockIdx.x;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
@@ -44,19 +66,20 @@ __global__ void __launch_bounds__(kQThreads)
     return;
   }
   const int rows = min(block, len - r0);
-  const int vpr = d / 8;  // 8 halves per 16-byte vector
   const int nv = rows * vpr;
   const size_t row_stride = static_cast<size_t>(heads) * d;
   const __half* base = x + (static_cast<size_t>(start + r0) * heads + h) * d;
 
-  uint4 v[kMaxVecs];
+  // Consecutive threads take consecutive 16-byte vectors of a row, so each
+  // row's VPR vectors are one coalesced read.
+  uint4 v[VPT];
   __half2 amax2 = __float2half2_rn(0.0f);
 #pragma unroll
-  for (int k = 0; k < kMaxVecs; ++k) {
+  for (int k = 0; k < VPT; ++k) {
     const int idx = threadIdx.x + k * kQThreads;
     if (idx < nv) {
       const int r = idx / vpr;
-      const int c = idx - r * vpr;
+      const int c = idx % vpr;
       v[k] = __ldg(reinterpret_cast<const uint4*>(base + r * row_stride) + c);
       const __half2* hv = reinterpret_cast<const __half2*>(&v[k]);
 #pragma unroll
@@ -75,29 +98,47 @@ __global__ void __launch_bounds__(kQThreads)
   for (int w = 1; w < kQThreads / 32; ++w) amax = fmaxf(amax, warp_max[w]);
 
   const float s = __fdiv_rn(amax, 127.0f);
+  const float rcp = amax != 0.0f ? __frcp_rn(s) : 0.0f;
   if (threadIdx.x == 0) *s_out = s;
   int8_t* qbase = x8 + (static_cast<size_t>(start + r0) * heads + h) * d;
 #pragma unroll
-  for (int k = 0; k < kMaxVecs; ++k) {
+  for (int k = 0; k < VPT; ++k) {
     const int idx = threadIdx.x + k * kQThreads;
     if (idx < nv) {
       const int r = idx / vpr;
-      const int c = idx - r * vpr;
+      const int c = idx % vpr;
       const __half* hv = reinterpret_cast<const __half*>(&v[k]);
       uint32_t packed[2] = {0u, 0u};
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        int q = 0;
-        if (amax != 0.0f) {
-          q = __float2int_rn(__fdiv_rn(__half2float(hv[e]), s));
-          q = max(-127, min(127, q));
-        }
+        const int q =
+            amax != 0.0f ? quant_code(__half2float(hv[e]), s, rcp) : 0;
         packed[e >> 2] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (e & 3));
       }
       *reinterpret_cast<uint2*>(qbase + r * row_stride + c * 8) =
           make_uint2(packed[0], packed[1]);
     }
   }
+}
+
+template <int VPR>
+cudaError_t launch_vpr(dim3 grid, int vecs, cudaStream_t stream,
+                       const __half* x, const int32_t* cu_seqlens, int batch,
+                       int max_seqlen, int total_tokens, int heads, int block,
+                       int nblk, int vpr_rt, int8_t* x8, float* scale,
+                       int32_t* status) {
+  const int vpt = (vecs + kQThreads - 1) / kQThreads;
+#define TILEMIX_QLAUNCH(N)                                                  \
+  quantize_kernel<N, VPR><<<grid, kQThreads, 0, stream>>>(                  \
+      x, cu_seqlens, batch, max_seqlen, total_tokens, heads, block, nblk,   \
+      vpr_rt, x8, scale, status)
+  if (vpt <= 2) TILEMIX_QLAUNCH(2);
+  else if (vpt <= 4) TILEMIX_QLAUNCH(4);
+  else if (vpt <= 8) TILEMIX_QLAUNCH(8);
+  else if (vpt <= 16) TILEMIX_QLAUNCH(16);
+  else return cudaErrorInvalidValue;
+#undef TILEMIX_QLAUNCH
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -110,10 +151,20 @@ cudaError_t launch_quantize_blockwise(const void* x, const int32_t* cu_seqlens,
                                       cudaStream_t stream) {
   const int nblk = (max_seqlen + block - 1) / block;
   dim3 grid(nblk, heads, batch);
-  quantize_kernel<<<grid, kQThreads, 0, stream>>>(
-      static_cast<const __half*>(x), cu_seqlens, batch, max_seqlen,
-      total_tokens, heads, head_dim, block, nblk, x8, scale, status);
-  return cudaGetLastError();
+  const __half* xh = static_cast<const __half*>(x);
+  const int vecs = block * head_dim / 8;
+  const int vpr = head_dim / 8;
+  if (head_dim == 128)
+    return launch_vpr<16>(grid, vecs, stream, xh, cu_seqlens, batch,
+                          max_seqlen, total_tokens, heads, block, nblk, vpr,
+                          x8, scale, status);
+  if (head_dim == 64)
+    return launch_vpr<8>(grid, vecs, stream, xh, cu_seqlens, batch,
+                         max_seqlen, total_tokens, heads, block, nblk, vpr, x8,
+                         scale, status);
+  return launch_vpr<0>(grid, vecs, stream, xh, cu_seqlens, batch, max_seqlen,
+                       total_tokens, heads, block, nblk, vpr, x8, scale,
+                       status);
 }
 
 }  // namespace tilemix
