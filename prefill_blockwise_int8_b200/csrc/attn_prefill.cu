@@ -11,23 +11,23 @@
 // B200 design.  A CTA owns kQT 128-row query tiles of one head of one
 // sequence (two tiles, rows 256M .. 256M+255; one tile with 64-row routing
 // words) and walks the 128-key compute tiles of their causal range:
-//   warp 8      TMA producer: Q and/or Q8 of its query tiles once, then per
+//   warp 16     TMA producer: Q and/or Q8 of its query tiles once, then per
 //               key tile the K tile in every format a query tile routes some
 //               of it to (fp16 and/or int8) and the fp16 V tile;
-//   warp 9      one thread issues tcgen05.mma: S_t = Q_t K^T (kind::f16, f32
+//   warp 17     one thread issues tcgen05.mma: S_t = Q_t K^T (kind::f16, f32
 //               in TMEM) or Q8_t K8^T (kind::i8, s32 in TMEM) per 64-key half
 //               of the tile (one N = 128 instruction chain when both halves
 //               take the same path), and O_t += P_t V with P_t read from TMEM
 //               (kind::f16, f32 TMEM accumulator);
-//   warps 0-7   softmax: with two query tiles, warps 0-3 serve tile 0 and
-//               warps 4-7 tile 1 (one thread per score row = TMEM lane), and
-//               the two warpgroups interleave on every SM sub-partition; with
-//               one query tile warps 0-3 take keys 0..63 and warps 4-7 keys
-//               64..127 of each row and combine row max and sum through
-//               shared memory.  Per tile: INT32 scores rescaled by
-//               q_scale * k_scale, causal / end-of-sequence masking, running
-//               max and sum in fp32, lazy rescale of O in TMEM when the max
-//               grows by more than 2^8, P back to TMEM as fp16; then O / l.
+//   warps 0-15  softmax: warpgroups 2t and 2t+1 serve query tile t, one
+//               thread per score row (= TMEM lane), keys 0..63 and 64..127
+//               of each row, combining row max and sum through shared
+//               memory; both tiles' warpgroups run at once, so every SM
+//               sub-partition holds four softmax warps.  Per tile: INT32
+//               scores rescaled by q_scale * k_scale, causal /
+//               end-of-sequence masking, running max and sum in fp32, lazy
+//               rescale of O in TMEM when the max grows by more than 2^8,
+//               P back to TMEM as fp16; then O / l.
 // 128-key tiles keep every FP16 MMA at N = 128: on sm_100a a kind::f16
 // M128 K16 instruction costs about the same at N = 64 as at N = 128.
 #include <cuda.h>
@@ -45,9 +45,9 @@ namespace {
 constexpr int kBM = 128;     // query rows per tile = TMEM lanes = MMA M
 constexpr int kBN = 128;     // keys per compute tile
 constexpr int kHalf = 64;    // routing granularity inside a compute tile
-constexpr int kWarpProducer = 8;
-constexpr int kWarpMma = 9;
-constexpr int kThreads = 320;
+constexpr int kWarpProducer = 16;
+constexpr int kWarpMma = 17;
+constexpr int kThreads = 576;
 constexpr int kSmemBudget = 232448;  // max dynamic smem per block on sm_100
 constexpr uint32_t kKindF16 = 1, kKindI8 = 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the
@@ -71,7 +71,7 @@ struct Cfg {
   static constexpr int kK8Off = align1k(kK16Bytes);
   static constexpr int kKSlotBytes = align1k(kK8Off + kK8Bytes);
   static constexpr int kVSlotBytes = align1k(kVBytes);
-  static constexpr int kRedBytes = 2048;  // row max / sum exchange [2][2][128]
+  static constexpr int kRedBytes = 4096;  // max / sum exchange [tile][2][2][128]
   static constexpr int kBarBytes = 512;
   static constexpr int kAvail =
       kSmemBudget - 1024 - kBarBytes - kRedBytes - kRing0;
@@ -110,8 +110,8 @@ struct Cfg {
   static constexpr int kBarS = kBarVEmpty + kVStages;  // [tile]
   static constexpr int kBarP = kBarS + 2;              // [tile]
   static constexpr int kBarO = kBarP + 2;              // [tile]
-  static constexpr int kBarRed = kBarO + 2;            // [parity]
-  static constexpr int kBarDrain = kBarRed + 2;
+  static constexpr int kBarRed = kBarO + 2;            // [tile][parity]
+  static constexpr int kBarDrain = kBarRed + 4;
   static constexpr int kNumBars = kBarDrain + 1;
   static_assert(kNumBars * 8 + 16 <= kBarBytes, "barrier area");
 };
@@ -176,6 +176,31 @@ __device__ __forceinline__ float max64(const uint32_t (&sv)[64], int hl) {
   }
 }
 
+// 2^x of a pair on the FMA and integer pipes, for the share of the
+// exponentials taken off the MUFU: x = j + f with j the nearest integer and
+// |f| <= 1/2; 2^f from a cubic fitted to 2^f on [-1/2, 1/2] by Remez
+// exchange (relative error <= 7.5e-5, below the fp16 rounding of P); 2^j
+// added to the exponent bits.  x is clamped to >= -125 so the result stays
+// normal (2^-125 stands for 0: it vanishes in fp16 and in the fp32 sums).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f,
+                  kC3 = 0.055171669f;
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = __fadd2_rn(x, make_float2(kIntBias, kIntBias));
+  const float2 j = __fadd2_rn(t, make_float2(-kIntBias, -kIntBias));
+  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
+  float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+  q = __ffma2_rn(q, f, make_float2(kC1, kC1));
+  q = __ffma2_rn(q, f, make_float2(kC0, kC0));
+  return make_float2(
+      __uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+      __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// Pairs of each 16-pair group computed by exp2_poly2 instead of the MUFU.
+constexpr int kPolyEvery = 4;
+
 // P = 2^(S c - m) of 32 scores as 16 packed fp16 pairs (key 2i in the low
 // half of pk[i]), added to four packed partial sums.  INT32 accumulators
 // convert to fp32 exactly (|acc| <= 127^2 d < 2^22) by the bias trick, on
@@ -208,7 +233,9 @@ __device__ __forceinline__ void exp32(const uint32_t (&sv)[32], float c,
       if (i & 1) xb = fmax3(xb, x.x, x.y);
       else xa = fmax3(xa, x.x, x.y);
     }
-    const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    const float2 pr = (i % kPolyEvery == kPolyEvery - 1)
+                          ? exp2_poly2(x)
+                          : make_float2(ex2_approx(x.x), ex2_approx(x.y));
     switch (i & 3) {
       case 0: ps0 = __fadd2_rn(ps0, pr); break;
       case 1: ps1 = __fadd2_rn(ps1, pr); break;
@@ -327,7 +354,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[C::kBarS + i], 1);
       mbar_init(&bars[C::kBarP + i], 8);   // one arrival per softmax warp
       mbar_init(&bars[C::kBarO + i], 1);
-      mbar_init(&bars[C::kBarRed + i], 8);
+      mbar_init(&bars[C::kBarRed + 2 * i], 8);
+      mbar_init(&bars[C::kBarRed + 2 * i + 1], 8);
     }
     mbar_init(&bars[C::kBarDrain], 1);
     *abort_flag = 0;
@@ -521,72 +549,67 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // =================== softmax warps 0-7 ===================
-    // Warpgroup wg takes keys 64*wg .. 64*wg+63 of every row (thread = row =
-    // TMEM lane) of each query tile.  Both warpgroups work on the CTA's
-    // query tiles one after the other (tile 0 then tile 1 for each key
-    // tile), so that one tile's softmax overlaps the other tile's P V and
-    // Q K^T on the tensor cores.  The row max is combined through shared
-    // memory every tile; each warpgroup keeps the sum of its own keys and
-    // the two are added once, at the end.
+    // =================== softmax warps 0-15 ===================
+    // Warpgroups 2t and 2t+1 serve query tile t: thread = score row = TMEM
+    // lane, warpgroup 2t + hw takes keys 64*hw .. 64*hw+63 of every row.  The
+    // two tiles' warpgroups run at the same time, one warp of each on every
+    // SM sub-partition, so one tile's latencies hide behind the other's
+    // arithmetic.  A tile's row max is combined by its two warpgroups
+    // through shared memory; each keeps the sum of its own keys and the two
+    // are added once, at the end.
     const int wg = warp >> 2;
+    const int t = wg >> 1;    // query tile
+    const int hw = wg & 1;    // key half
     const int r = threadIdx.x & 127;
-    const int c0 = wg * kHalf;  // first key of this thread inside a key tile
+    const int c0 = hw * kHalf;  // first key of this thread inside a key tile
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const float* kscale =
-        routed ? p.k_scale + (static_cast<size_t>(hk) * p.batch + b) * p.nbk
-               : nullptr;
-    // K scale of this thread's 64 keys; the next key tile's is fetched while
-    // the current one is processed.
-    auto ksc = [&](int n) {
-      const int blk = (n * kBN + c0) / p.quant_block_k;
-      return kscale[min(blk, p.nbk - 1)];
-    };
-    float sk_next = routed ? ksc(0) : 0.0f;
-    // softmax scale (log2 units) times the Q block scale of this thread's row
-    // in each query tile: the INT8 path's S c = (Q8 K8^T) sq sk scale log2(e)
-    auto qsc = [&](int t) {
-      const int key_lim = min(row_base + t * kBM + r, len - 1);
-      return (routed && key_lim >= 0)
-                 ? p.scale_log2 *
+    bool ok = true;
+    if (t < kQT) {
+      const TileRoute& R = rt(t);
+      const int r_local = row_base + t * kBM + r;
+      const int rh = DUAL ? (r >> 6) : 0;  // routing row half
+      const uint64_t my_w = rh ? R.w1 : R.w0;
+      const int my_nl = rh ? R.nl1 : R.nl0;
+      const int key_lim = min(r_local, len - 1);  // keys j <= key_lim legal
+      const uint32_t lane_addr = tmem + t * C::kTileCols + lane_off;
+      const float* kscale =
+          routed ? p.k_scale + (static_cast<size_t>(hk) * p.batch + b) * p.nbk
+                 : nullptr;
+      // K scale of this thread's 64 keys; the next key tile's is fetched
+      // while the current one is processed.
+      auto ksc = [&](int n) {
+        const int blk = (n * kBN + c0) / p.quant_block_k;
+        return kscale[min(blk, p.nbk - 1)];
+      };
+      float sk_next = (routed && R.n_last >= 0) ? ksc(0) : 0.0f;
+      // softmax scale (log2 units) times the Q block scale of this row: the
+      // INT8 path's S c = (Q8 K8^T) sq sk scale log2(e)
+      const float cq =
+          routed ? p.scale_log2 *
                        p.q_scale[(static_cast<size_t>(h) * p.batch + b) * p.nbq +
                                  key_lim / p.quant_block_q]
                  : 0.0f;
-    };
-    const float cq0 = qsc(0), cq1 = kQT > 1 ? qsc(1) : 0.0f;
-    // running max and (this warpgroup's) sum of each query tile's rows
-    float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.0f, l1 = 0.0f;
-    uint32_t u = 0;  // tiles processed so far: parity of the exchange slot
-    bool ok = true;
-    // Combine a per-row value with the other warpgroup's (max or sum).
-    auto exchange = [&](float v, bool& good) -> float {
-      float* slot = red + (u & 1) * 256;
-      slot[wg * 128 + r] = v;
-      __syncwarp();  // orders the lanes' stores before lane 0's release
-      if (lane == 0) mbar_arrive(&bars[C::kBarRed + (u & 1)]);
-      const bool got = mbar_wait(&bars[C::kBarRed + (u & 1)], (u >> 1) & 1,
-                                 abort_flag);
-      good = __all_sync(0xffffffffu, got);
-      const float other = slot[(1 - wg) * 128 + r];
-      ++u;
-      return other;
-    };
+      // running max and (this warpgroup's) sum of the row
+      float m_run = -CUDART_INF_F, l_run = 0.0f;
+      uint32_t u = 0;  // exchanges so far: slot and parity
+      float* red_t = red + t * 512;
+      uint64_t* bar_red = &bars[C::kBarRed + 2 * t];
+      // Combine a per-row value with the other warpgroup's (max or sum).
+      auto exchange = [&](float v, bool& good) -> float {
+        float* slot = red_t + (u & 1) * 256;
+        slot[hw * 128 + r] = v;
+        __syncwarp();  // orders the lanes' stores before lane 0's release
+        if (lane == 0) mbar_arrive(&bar_red[u & 1]);
+        const bool got = mbar_wait(&bar_red[u & 1], (u >> 1) & 1, abort_flag);
+        good = __all_sync(0xffffffffu, got);
+        const float other = slot[(1 - hw) * 128 + r];
+        ++u;
+        return other;
+      };
 
-    for (int n = 0; n <= n_end && ok; ++n) {
-      const float sk = sk_next;
-      if (routed && n < n_end) sk_next = ksc(n + 1);
-#pragma unroll 1
-      for (int t = 0; t < kQT; ++t) {
-        const TileRoute& R = rt(t);
-        if (n > R.n_last) continue;  // same decision in both warpgroups
-        const int r_local = row_base + t * kBM + r;
-        const int rh = DUAL ? (r >> 6) : 0;  // routing row half
-        const uint64_t my_w = rh ? R.w1 : R.w0;
-        const int my_nl = rh ? R.nl1 : R.nl0;
-        const int key_lim = min(r_local, len - 1);  // keys j <= key_lim legal
-        const uint32_t tb = tmem + t * C::kTileCols;
-        const uint32_t lane_addr = tb + lane_off;
-
+      for (int n = 0; n <= R.n_last; ++n) {
+        const float sk = sk_next;
+        if (routed && n < R.n_last) sk_next = ksc(n + 1);
         // Exits stay warp-uniform: the tcgen05.ld/st below are .sync.aligned.
         const bool got_s = mbar_wait(&bars[C::kBarS + t], n & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got_s)) {
@@ -597,41 +620,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Path of this thread's 64 keys for its routing row half.  Keys past
         // every row of the tile: the MMA wrote the first half's path there
         // (values masked below either way).
-        const int n64 = 2 * n + wg;
+        const int n64 = 2 * n + hw;
         const int nb = (!DUAL && n64 > my_nl) ? 2 * n : n64;
         const bool i8 =
             (nb <= my_nl) && (((my_w >> (nb / tpb)) & 1ull) != 0);
-        const float c = i8 ? (t ? cq1 : cq0) * sk : p.scale_log2;
-        uint32_t sv[kHalf];
+        const float c = i8 ? cq * sk : p.scale_log2;
         const uint32_t scol = lane_addr + (i8 ? C::kS8 : C::kS16) + c0;
-        tmem_ld32(scol, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld_wait();
-        if (p.qk_dump && r_local < len && i8 && n64 <= my_nl) {
-          const int rrow = r_local / p.route_bm;
-          const int rr = r_local - rrow * p.route_bm;
-          const int key0 = n64 * kHalf;
-          const int nr = key0 / p.route_bn;
-          int32_t* dst =
-              p.qk_dump +
-              ((((static_cast<size_t>(b) * p.hq + h) * p.tm_route + rrow) *
-                    p.tn_max +
-                nr) *
-                   p.route_bm +
-               rr) *
-                  p.route_bn +
-              (key0 - nr * p.route_bn);
-          const int keys_left = len - key0;  // keys inside the sequence
-#pragma unroll
-          for (int j = 0; j < kHalf; ++j)
-            if (j < keys_left) dst[j] = static_cast<int32_t>(sv[j]);
-        }
         const int hl = key_lim - n * kBN - c0;  // legal columns: j <= hl
-        const bool fullh = hl >= kHalf - 1;
-        const float mx = i8 ? (fullh ? max64<true, false>(sv, hl)
-                                     : max64<true, true>(sv, hl))
-                            : (fullh ? max64<false, false>(sv, hl)
-                                     : max64<false, true>(sv, hl));
+        float mx;
+        {  // pass 1: the 64 scores only live for the row max
+          uint32_t sv[kHalf];
+          tmem_ld32(scol, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_ld_wait();
+          if (p.qk_dump && r_local < len && i8 && n64 <= my_nl) {
+            const int rrow = r_local / p.route_bm;
+            const int rr = r_local - rrow * p.route_bm;
+            const int key0 = n64 * kHalf;
+            const int nr = key0 / p.route_bn;
+            int32_t* dst =
+                p.qk_dump +
+                ((((static_cast<size_t>(b) * p.hq + h) * p.tm_route + rrow) *
+                      p.tn_max +
+                  nr) *
+                     p.route_bm +
+                 rr) *
+                    p.route_bn +
+                (key0 - nr * p.route_bn);
+            const int keys_left = len - key0;  // keys inside the sequence
+  #pragma unroll
+            for (int j = 0; j < kHalf; ++j)
+              if (j < keys_left) dst[j] = static_cast<int32_t>(sv[j]);
+        }
+          const bool fullh = hl >= kHalf - 1;
+          mx = i8 ? (fullh ? max64<true, false>(sv, hl)
+                           : max64<true, true>(sv, hl))
+                  : (fullh ? max64<false, false>(sv, hl)
+                           : max64<false, true>(sv, hl));
+        }
         const float m_half = (mx == -CUDART_INF_F) ? -CUDART_INF_F : mx * c;
         bool good = true;
         const float m_tile = fmaxf(m_half, exchange(m_half, good));
@@ -639,42 +665,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        float m_run = t ? m1 : m0;
-        float l_run = t ? l1 : l0;
-        const float m_new = fmaxf(m_run, m_tile);
-        const bool need = m_new > m_run + kRescaleThreshold;
+        // Lazy rescaling: keep the old max unless the tile exceeds it by
+        // more than 2^threshold, so P <= 2^threshold stays in fp16 range.
+        const bool need = m_tile > m_run + kRescaleThreshold;
         const float m_old = m_run;
         if (need) {
-          l_run *= ex2_approx(m_run - m_new);
-          m_run = m_new;
+          l_run *= ex2_approx(m_run - m_tile);
+          m_run = m_tile;
         }
         // P = 2^(S c - m) of this thread's 64 keys as fp16 pairs over the S
         // columns it has just read (key 2i in the low half of column i).
         float2 ps0 = make_float2(0.f, 0.f), ps1 = ps0, ps2 = ps0, ps3 = ps0;
         float unused_max = 0.0f;
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < 2; ++q) {  // pass 2: reload 32 scores at a time
+          uint32_t sq32[32];
+          tmem_ld32(scol + 32 * q, sq32);
+          tmem_ld_wait();
           uint32_t pk[16];
           const int hq = hl - 32 * q;
-          const uint32_t(&sq32)[32] =
-              *reinterpret_cast<const uint32_t(*)[32]>(&sv[32 * q]);
-          uint32_t* pkq = pk;
           const bool fullq = hq >= 31;
           if (i8) {
-            if (fullq) exp32<true, false, false>(sq32, c, m_run, hq, pkq, ps0, ps1, ps2, ps3, unused_max);
-            else exp32<true, true, false>(sq32, c, m_run, hq, pkq, ps0, ps1, ps2, ps3, unused_max);
+            if (fullq) exp32<true, false, false>(sq32, c, m_run, hq, pk, ps0, ps1, ps2, ps3, unused_max);
+            else exp32<true, true, false>(sq32, c, m_run, hq, pk, ps0, ps1, ps2, ps3, unused_max);
           } else {
-            if (fullq) exp32<false, false, false>(sq32, c, m_run, hq, pkq, ps0, ps1, ps2, ps3, unused_max);
-            else exp32<false, true, false>(sq32, c, m_run, hq, pkq, ps0, ps1, ps2, ps3, unused_max);
+            if (fullq) exp32<false, false, false>(sq32, c, m_run, hq, pk, ps0, ps1, ps2, ps3, unused_max);
+            else exp32<false, true, false>(sq32, c, m_run, hq, pk, ps0, ps1, ps2, ps3, unused_max);
           }
-          tmem_st16(lane_addr + C::p_col(wg) + 16 * q, pk);
+          tmem_st16(lane_addr + C::p_col(hw) + 16 * q, pk);
         }
         if (n > 0 && __any_sync(0xffffffffu, need)) {
           // S_t(n) is ready, so P V_t(n-1) completed (the MMA thread issues
           // Q K^T_t(n) after it): O_t can be rescaled now.  Each warpgroup
           // rescales half of O's columns.
-          const float alpha = need ? ex2_approx(m_old - m_new) : 1.0f;
-          const int o0 = wg * (D / 2);
+          const float alpha = need ? ex2_approx(m_old - m_tile) : 1.0f;
+          const int o0 = hw * (D / 2);
 #pragma unroll
           for (int oc = 0; oc < D / 2; oc += 32) {
             uint32_t o[32];
@@ -688,69 +713,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float2 s4 = __fadd2_rn(__fadd2_rn(ps0, ps1), __fadd2_rn(ps2, ps3));
         l_run += s4.x + s4.y;
-        if (t) {
-          m1 = m_run;
-          l1 = l_run;
-        } else {
-          m0 = m_run;
-          l0 = l_run;
-        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[C::kBarP + t]);
       }
-    }
 
-    // Epilogue of each query tile: O / l, both warpgroups' sums combined;
-    // each warpgroup stores half of O's columns.
-#pragma unroll 1
-    for (int t = 0; t < kQT; ++t) {
-      const TileRoute& R = rt(t);
-      if (R.n_last < 0) continue;
-      const bool got_last =
-          ok && mbar_wait(&bars[C::kBarO + t], R.n_last & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, got_last)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      bool good = true;
-      const float l_mine = t ? l1 : l0;
-      const float l_run = l_mine + exchange(l_mine, good);
-      if (!good) {
-        ok = false;
-        break;
-      }
-      const float m_run = t ? m1 : m0;
-      const int r_local = row_base + t * kBM + r;
-      const bool valid = r_local < len;
-      const uint32_t lane_addr = tmem + t * C::kTileCols + lane_off;
-      const float inv_l = 1.0f / l_run;
-      const int o0 = wg * (D / 2);
-      uint16_t* orow =
-          p.out + (static_cast<size_t>(start + r_local) * p.hq + h) * D + o0;
+      // Epilogue: O / l with both warpgroups' sums; each warpgroup stores
+      // half of O's columns.
+      if (ok && R.n_last >= 0) {
+        const bool got_last =
+            mbar_wait(&bars[C::kBarO + t], R.n_last & 1, abort_flag);
+        ok = __all_sync(0xffffffffu, got_last);
+        if (ok) {
+          tc_fence_after();
+          bool good = true;
+          const float l_tot = l_run + exchange(l_run, good);
+          ok = good;
+          if (ok) {
+            const bool valid = r_local < len;
+            const float inv_l = 1.0f / l_tot;
+            const int o0 = hw * (D / 2);
+            uint16_t* orow =
+                p.out + (static_cast<size_t>(start + r_local) * p.hq + h) * D +
+                o0;
 #pragma unroll
-      for (int oc = 0; oc < D / 2; oc += 32) {
-        uint32_t o[32];
-        tmem_ld32(lane_addr + C::kOCol + o0 + oc, o);
-        tmem_ld_wait();
-        uint32_t hv[16];
+            for (int oc = 0; oc < D / 2; oc += 32) {
+              uint32_t o[32];
+              tmem_ld32(lane_addr + C::kOCol + o0 + oc, o);
+              tmem_ld_wait();
+              uint32_t hv[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          hv[j] = pack_half2(__uint_as_float(o[2 * j]) * inv_l,
-                             __uint_as_float(o[2 * j + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + oc);
+              for (int j = 0; j < 16; ++j)
+                hv[j] = pack_half2(__uint_as_float(o[2 * j]) * inv_l,
+                                   __uint_as_float(o[2 * j + 1]) * inv_l);
+              if (valid) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + oc);
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(hv[4 * v], hv[4 * v + 1], hv[4 * v + 2],
-                                hv[4 * v + 3]);
+                for (int v = 0; v < 4; ++v)
+                  dst[v] = make_uint4(hv[4 * v], hv[4 * v + 1], hv[4 * v + 2],
+                                      hv[4 * v + 3]);
+              }
+            }
+            if (p.lse && valid && hw == 0)
+              p.lse[static_cast<size_t>(h) * p.total_tokens + start + r_local] =
+                  (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
+          }
         }
       }
-      if (p.lse && valid && wg == 0)
-        p.lse[static_cast<size_t>(h) * p.total_tokens + start + r_local] =
-            (m_run + __log2f(l_run)) * 0.69314718055994530942f;
     }
     if (!ok) fail();
   }
