@@ -47,7 +47,9 @@ constexpr int kBN = 128;     // keys per compute tile
 constexpr int kHalf = 64;    // routing granularity inside a compute tile
 constexpr int kWarpProducer = 16;
 constexpr int kWarpMma = 17;
-constexpr int kThreads = 576;
+constexpr int kWarpConv = 18;  // two warps, INT8 KV cache only
+// 16 softmax warps, producer, MMA issuer (+ two converter warps)
+__host__ __device__ constexpr int threads_of(bool kv8) { return kv8 ? 640 : 576; }
 constexpr int kSmemBudget = 232448;  // max dynamic smem per block on sm_100
 constexpr uint32_t kKindF16 = 1, kKindI8 = 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the
@@ -55,7 +57,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the
 
 __host__ __device__ constexpr int align1k(int x) { return (x + 1023) & ~1023; }
 
-template <int D, bool DUAL>
+template <int D, bool DUAL, bool KV8>
 struct Cfg {
   // DUAL (64-row routing words): a 128-row query tile may need both paths
   // for the same keys, so S has an fp16 and an int8 region and the CTA
@@ -66,11 +68,18 @@ struct Cfg {
   static constexpr int kK16Bytes = kBN * D * 2;
   static constexpr int kK8Bytes = kBN * D;
   static constexpr int kVBytes = kBN * D * 2;
+  // INT8 V tile, staged in the upper half of its V slot and converted in
+  // place (row r of V8 lies exactly where chunk D/64 - 1 of row r of V goes
+  // for d = 128; rows are converted by the thread that read them)
+  static constexpr int kV8Bytes = kBN * D;
+  static constexpr int kV8Off = D == 128 ? kVBytes - kV8Bytes : kVBytes;
   static constexpr int kQ8Off = kQT * kQBytes;
   static constexpr int kRing0 = align1k(kQ8Off + kQT * kQ8Bytes);
   static constexpr int kK8Off = align1k(kK16Bytes);
   static constexpr int kKSlotBytes = align1k(kK8Off + kK8Bytes);
-  static constexpr int kVSlotBytes = align1k(kVBytes);
+  // (d = 64 stages V8 past the fp16 tile: there rows would overlap)
+  static constexpr int kVSlotBytes =
+      align1k(KV8 && D != 128 ? kVBytes + kBN * D : kVBytes);
   static constexpr int kRedBytes = 4096;  // max / sum exchange [tile][2][2][128]
   static constexpr int kBarBytes = 512;
   static constexpr int kAvail =
@@ -111,7 +120,10 @@ struct Cfg {
   static constexpr int kBarP = kBarS + 2;              // [tile]
   static constexpr int kBarO = kBarP + 2;              // [tile]
   static constexpr int kBarRed = kBarO + 2;            // [tile][parity]
-  static constexpr int kBarDrain = kBarRed + 4;
+  // INT8 KV cache: K slot holds its fp16 copy, V slot its fp16 V
+  static constexpr int kBarKConv = kBarRed + 4;        // [K slot]
+  static constexpr int kBarVConv = kBarKConv + kKStages;  // [V slot]
+  static constexpr int kBarDrain = kBarVConv + kVStages;
   static constexpr int kNumBars = kBarDrain + 1;
   static_assert(kNumBars * 8 + 16 <= kBarBytes, "barrier area");
 };
@@ -247,6 +259,65 @@ __device__ __forceinline__ void exp32(const uint32_t (&sv)[32], float c,
   if (TRACK) xmax = fmax3(xmax, xa, xb);
 }
 
+// Byte offset inside a tile stored with the 128- (m = 7) or 64-byte (m = 3)
+// swizzle: 16-byte unit bits [4:6] XOR row bits [7:9].
+__device__ __forceinline__ uint32_t swz(uint32_t o, uint32_t m) {
+  return o ^ (((o >> 7) & m) << 4);
+}
+
+// Four int8 (one word) -> two fp16 pairs, exactly: bias the bytes to
+// unsigned, place each under the fp16 exponent of 1024 (0x64xx = 1024 +
+// byte), subtract 1024 + 128.
+__device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo,
+                                             uint32_t& hi) {
+  const uint32_t x = w ^ 0x80808080u;
+  const __half2 bias = __float2half2_rn(1152.0f);
+  uint32_t a = __byte_perm(x, 0x64646464u, 0x4140);
+  uint32_t b = __byte_perm(x, 0x64646464u, 0x4342);
+  __half2 ha = __hsub2(*reinterpret_cast<__half2*>(&a), bias);
+  __half2 hb = __hsub2(*reinterpret_cast<__half2*>(&b), bias);
+  lo = *reinterpret_cast<uint32_t*>(&ha);
+  hi = *reinterpret_cast<uint32_t*>(&hb);
+}
+
+// One key row of an INT8 tile (D bytes at row rr of `src`, swizzled with
+// mask sm, 0 = plain rows) -> the fp16 K-major / V layout: D/64 chunks of
+// [128 rows][128 B] with the 128-byte swizzle.  With SCALE, each value is
+// multiplied by s2 (rounded once to fp16).  The whole row is read before
+// any store, so the fp16 row may overlap the INT8 row it came from.
+template <int D, bool SCALE>
+__device__ __forceinline__ void convert_row(const uint8_t* src, uint32_t sm,
+                                            uint8_t* dst, int rr,
+                                            __half2 s2) {
+  uint4 in[D / 16];
+#pragma unroll
+  for (int u = 0; u < D / 16; ++u)
+    in[u] = *reinterpret_cast<const uint4*>(src + swz(rr * D + u * 16, sm));
+#pragma unroll
+  for (int u = 0; u < D / 16; ++u) {
+    const uint32_t w[4] = {in[u].x, in[u].y, in[u].z, in[u].w};
+    uint32_t h[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) i8x4_to_h2x2(w[i], h[2 * i], h[2 * i + 1]);
+    if (SCALE) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        __half2 v = __hmul2(*reinterpret_cast<__half2*>(&h[i]), s2);
+        h[i] = *reinterpret_cast<uint32_t*>(&v);
+      }
+    }
+    // dims 16u .. 16u+15 -> chunk (16u) / 64, 16-byte units 2u, 2u+1 of it
+    const int c = (16 * u) / 64;
+    const int uo = (2 * u) % 8;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const uint32_t o = c * 128 * 128 + rr * 128 + (uo + e) * 16;
+      *reinterpret_cast<uint4*>(dst + swz(o, 7)) =
+          make_uint4(h[4 * e], h[4 * e + 1], h[4 * e + 2], h[4 * e + 3]);
+    }
+  }
+}
+
 // Routing state of one 128-row query tile.
 struct TileRoute {
   uint64_t w0, w1;  // words of rows 0..63 / 64..127 (equal unless DUAL)
@@ -254,10 +325,10 @@ struct TileRoute {
   int n_last;       // last legal 128-key tile (-1: no rows)
 };
 
-template <int D, bool DUAL>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, bool DUAL, bool KV8>
+__global__ void __launch_bounds__(threads_of(KV8), 1)
     attn_fwd_kernel(const __grid_constant__ AttnParams p) {
-  using C = Cfg<D, DUAL>;
+  using C = Cfg<D, DUAL, KV8>;
   constexpr int kQT = C::kQT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -357,15 +428,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[C::kBarRed + 2 * i], 8);
       mbar_init(&bars[C::kBarRed + 2 * i + 1], 8);
     }
+    if (KV8) {
+      for (int s = 0; s < C::kKStages; ++s)
+        mbar_init(&bars[C::kBarKConv + s], 2);  // the two converter warps
+      for (int s = 0; s < C::kVStages; ++s)
+        mbar_init(&bars[C::kBarVConv + s], 2);
+    }
     mbar_init(&bars[C::kBarDrain], 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&p.tm_q);
-    tma_prefetch_desc(&p.tm_k);
-    tma_prefetch_desc(&p.tm_v);
+    if (KV8) {
+      tma_prefetch_desc(&p.tm_k8);
+      tma_prefetch_desc(&p.tm_v8);
+    } else {
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+    }
     if (routed) {  // the INT8 maps are left empty in FP16-only mode
       tma_prefetch_desc(&p.tm_q8);
-      tma_prefetch_desc(&p.tm_k8);
+      if (!KV8) tma_prefetch_desc(&p.tm_k8);
     }
   }
   if (warp == kWarpMma) {
@@ -418,6 +500,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t kinds = 0;
         for (int t = 0; t < kQT; ++t)
           kinds |= kinds_of(t, n, 0) | kinds_of(t, n, 1);
+        // The INT8 cache only holds K8 (the converters make the fp16 copy).
+        if (KV8) kinds = kKindI8;
         mbar_arrive_expect_tx(&bars[C::kBarK + ks],
                               ((kinds & kKindF16) ? C::kK16Bytes : 0) +
                                   ((kinds & kKindI8) ? C::kK8Bytes : 0));
@@ -437,10 +521,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&bars[C::kBarV + vs], C::kVBytes);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(vslot(vs) + c * kBN * 128, &p.tm_v, &bars[C::kBarV + vs],
-                      c * 64, krow, hk);
+        if (KV8) {
+          mbar_arrive_expect_tx(&bars[C::kBarV + vs], C::kV8Bytes);
+          tma_load_3d(vslot(vs) + C::kV8Off, &p.tm_v8, &bars[C::kBarV + vs], 0,
+                      krow, hk);
+        } else {
+          mbar_arrive_expect_tx(&bars[C::kBarV + vs], C::kVBytes);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(vslot(vs) + c * kBN * 128, &p.tm_v,
+                        &bars[C::kBarV + vs], c * 64, krow, hk);
+        }
         v_issued = n + 1;
       }
       if (!ok) {
@@ -482,6 +572,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   ((k1 & kKindF16) ? 2u : 0u);
         const uint32_t halves8 = ((k0 & kKindI8) ? 1u : 0u) |
                                  ((k1 & kKindI8) ? 2u : 0u);
+        if (halves16 && KV8 &&
+            !mbar_wait(&bars[C::kBarKConv + s], (n / C::kKStages) & 1,
+                       abort_flag))
+          return false;
         if (halves16) {
           const uint32_t q16 = smem_u32(sQ(t));
           const bool both = halves16 == 3u;
@@ -513,7 +607,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (n > rt(t).n_last) return true;
         const int s = n % C::kVStages;
         if (!mbar_wait(&bars[C::kBarP + t], n & 1, abort_flag)) return false;
-        if (!mbar_wait(&bars[C::kBarV + s], (n / C::kVStages) & 1, abort_flag))
+        // INT8 cache: the converters' fp16 V (they waited for the TMA)
+        if (!mbar_wait(&bars[(KV8 ? C::kBarVConv : C::kBarV) + s],
+                       (n / C::kVStages) & 1, abort_flag))
           return false;
         tc_fence_after();
         const uint32_t vb = smem_u32(vslot(s));
@@ -548,6 +644,67 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&bars[C::kBarDrain], 0, nullptr);
     }
     __syncwarp();
+  } else if (warp >= kWarpConv) {
+    // =================== INT8 KV cache converters (2 warps) ===================
+    // Per key tile: K8 -> fp16 K (exact; only when some query tile routes
+    // part of the tile to FP16) and V8 -> fp16 v8 * v_scale.  Each thread
+    // converts whole key rows (rows ct and ct + 64), reading a row before
+    // writing it, which makes the in-place V conversion safe.
+    if (KV8) {
+      const int ct = (warp - kWarpConv) * 32 + lane;
+      const float* vscale =
+          p.v_scale + (static_cast<size_t>(hk) * p.batch + b) * p.nbk;
+      constexpr uint32_t k8_swz = D == 128 ? 7u : 3u;
+      bool ok = true;
+      for (int n = 0; n <= n_end && ok; ++n) {
+        const int ks = n % C::kKStages;
+        const bool got_k = mbar_wait(&bars[C::kBarK + ks],
+                                     (n / C::kKStages) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got_k)) {
+          ok = false;
+          break;
+        }
+        uint32_t kinds = 0;
+        for (int t = 0; t < kQT; ++t)
+          kinds |= kinds_of(t, n, 0) | kinds_of(t, n, 1);
+        if (kinds & kKindF16) {
+          uint8_t* kslot_p = kslot(ks);
+#pragma unroll 1
+          for (int rr = ct; rr < kBN; rr += 64)
+            convert_row<D, false>(kslot_p + C::kK8Off, k8_swz, kslot_p, rr,
+                                  __float2half2_rn(1.0f));
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[C::kBarKConv + ks]);
+
+        const int vs = n % C::kVStages;
+        const bool got_v = mbar_wait(&bars[C::kBarV + vs],
+                                     (n / C::kVStages) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got_v)) {
+          ok = false;
+          break;
+        }
+        uint8_t* vslot_p = vslot(vs);
+#pragma unroll 1
+        for (int rr = ct; rr < kBN; rr += 64) {
+          // V scale sv = 2^e2 f with f in [1, 2): the fp16 tile holds
+          // v8 2^e2 exactly (never above |v8 sv|); the softmax multiplies P
+          // by f.
+          const int blk = (n * kBN + rr) / p.quant_block_k;
+          const float sv = vscale[min(blk, p.nbk - 1)];
+          int e = 0;
+          frexpf(sv, &e);
+          const float pow2 = sv > 0.0f ? ldexpf(1.0f, e - 1) : 0.0f;
+          convert_row<D, true>(vslot_p + C::kV8Off, 0u, vslot_p, rr,
+                               __float2half2_rn(pow2));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[C::kBarVConv + vs]);
+      }
+      if (!ok) fail();
+    }
   } else {
     // =================== softmax warps 0-15 ===================
     // Warpgroups 2t and 2t+1 serve query tile t: thread = score row = TMEM
@@ -573,15 +730,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int key_lim = min(r_local, len - 1);  // keys j <= key_lim legal
       const uint32_t lane_addr = tmem + t * C::kTileCols + lane_off;
       const float* kscale =
-          routed ? p.k_scale + (static_cast<size_t>(hk) * p.batch + b) * p.nbk
-                 : nullptr;
+          (routed || KV8)
+              ? p.k_scale + (static_cast<size_t>(hk) * p.batch + b) * p.nbk
+              : nullptr;
       // K scale of this thread's 64 keys; the next key tile's is fetched
       // while the current one is processed.
       auto ksc = [&](int n) {
         const int blk = (n * kBN + c0) / p.quant_block_k;
         return kscale[min(blk, p.nbk - 1)];
       };
-      float sk_next = (routed && R.n_last >= 0) ? ksc(0) : 0.0f;
+      float sk_next = ((routed || KV8) && R.n_last >= 0) ? ksc(0) : 0.0f;
+      // INT8 KV cache: the V scale's mantissa factor f in [1, 2) of this
+      // thread's 64 keys (the converters put its power of two into V).
+      const float* vscale =
+          KV8 ? p.v_scale + (static_cast<size_t>(hk) * p.batch + b) * p.nbk
+              : nullptr;
+      auto vfrac = [&](int n) {
+        const int blk = (n * kBN + c0) / p.quant_block_k;
+        const float sv = vscale[min(blk, p.nbk - 1)];
+        int e = 0;
+        frexpf(sv, &e);
+        return sv > 0.0f ? ldexpf(sv, 1 - e) : 1.0f;
+      };
+      float fv_next = (KV8 && R.n_last >= 0) ? vfrac(0) : 1.0f;
       // softmax scale (log2 units) times the Q block scale of this row: the
       // INT8 path's S c = (Q8 K8^T) sq sk scale log2(e)
       const float cq =
@@ -609,7 +780,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       for (int n = 0; n <= R.n_last; ++n) {
         const float sk = sk_next;
-        if (routed && n < R.n_last) sk_next = ksc(n + 1);
+        if ((routed || KV8) && n < R.n_last) sk_next = ksc(n + 1);
+        const float fv = fv_next;
+        if (KV8 && n < R.n_last) fv_next = vfrac(n + 1);
         // Exits stay warp-uniform: the tcgen05.ld/st below are .sync.aligned.
         const bool got_s = mbar_wait(&bars[C::kBarS + t], n & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got_s)) {
@@ -624,7 +797,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nb = (!DUAL && n64 > my_nl) ? 2 * n : n64;
         const bool i8 =
             (nb <= my_nl) && (((my_w >> (nb / tpb)) & 1ull) != 0);
-        const float c = i8 ? cq * sk : p.scale_log2;
+        // FP16 keys of the INT8 cache are k8 exactly: their scale joins c.
+        const float c = i8 ? cq * sk : (KV8 ? p.scale_log2 * sk : p.scale_log2);
         const uint32_t scol = lane_addr + (i8 ? C::kS8 : C::kS16) + c0;
         const int hl = key_lim - n * kBN - c0;  // legal columns: j <= hl
         float mx;
@@ -677,6 +851,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // columns it has just read (key 2i in the low half of column i).
         float2 ps0 = make_float2(0.f, 0.f), ps1 = ps0, ps2 = ps0, ps3 = ps0;
         float unused_max = 0.0f;
+        // INT8 KV cache: P f = 2^(S c - m + log2 f) goes to the P V product
+        // (<= 2^9, fp16-safe); the row sum divides f out again.
+        const float m_exp = KV8 ? m_run - __log2f(fv) : m_run;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {  // pass 2: reload 32 scores at a time
           uint32_t sq32[32];
@@ -686,11 +863,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int hq = hl - 32 * q;
           const bool fullq = hq >= 31;
           if (i8) {
-            if (fullq) exp32<true, false, false>(sq32, c, m_run, hq, pk, ps0, ps1, ps2, ps3, unused_max);
-            else exp32<true, true, false>(sq32, c, m_run, hq, pk, ps0, ps1, ps2, ps3, unused_max);
+            if (fullq) exp32<true, false, false>(sq32, c, m_exp, hq, pk, ps0, ps1, ps2, ps3, unused_max);
+            else exp32<true, true, false>(sq32, c, m_exp, hq, pk, ps0, ps1, ps2, ps3, unused_max);
           } else {
-            if (fullq) exp32<false, false, false>(sq32, c, m_run, hq, pk, ps0, ps1, ps2, ps3, unused_max);
-            else exp32<false, true, false>(sq32, c, m_run, hq, pk, ps0, ps1, ps2, ps3, unused_max);
+            if (fullq) exp32<false, false, false>(sq32, c, m_exp, hq, pk, ps0, ps1, ps2, ps3, unused_max);
+            else exp32<false, true, false>(sq32, c, m_exp, hq, pk, ps0, ps1, ps2, ps3, unused_max);
           }
           tmem_st16(lane_addr + C::p_col(hw) + 16 * q, pk);
         }
@@ -712,7 +889,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const float2 s4 = __fadd2_rn(__fadd2_rn(ps0, ps1), __fadd2_rn(ps2, ps3));
-        l_run += s4.x + s4.y;
+        l_run += KV8 ? (s4.x + s4.y) / fv : s4.x + s4.y;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -771,37 +948,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpMma) tmem_dealloc(tmem, C::kTmemCols);
 }
 
-template <int D, bool DUAL>
+template <int D, bool DUAL, bool KV8>
 cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
-  using C = Cfg<D, DUAL>;
-  auto kern = attn_fwd_kernel<D, DUAL>;
+  using C = Cfg<D, DUAL, KV8>;
+  auto kern = attn_fwd_kernel<D, DUAL, KV8>;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const int groups = (p.max_seqlen + C::kQT * kBM - 1) / (C::kQT * kBM);
   dim3 grid(p.hq, groups, p.batch);
-  kern<<<grid, kThreads, C::kSmem, stream>>>(p);
+  kern<<<grid, threads_of(KV8), C::kSmem, stream>>>(p);
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const AttnParams& p, const AttnLaunchShape& s,
+                     cudaStream_t stream) {
+  if (s.kv8)
+    return s.dual ? launch_one<D, true, true>(p, stream)
+                  : launch_one<D, false, true>(p, stream);
+  return s.dual ? launch_one<D, true, false>(p, stream)
+                : launch_one<D, false, false>(p, stream);
+}
+
+template <int D>
+int smem_d(const AttnLaunchShape& s) {
+  if (s.kv8)
+    return s.dual ? Cfg<D, true, true>::kSmem : Cfg<D, false, true>::kSmem;
+  return s.dual ? Cfg<D, true, false>::kSmem : Cfg<D, false, false>::kSmem;
 }
 
 }  // namespace
 
 cudaError_t launch_attn_prefill(const AttnParams& p, const AttnLaunchShape& s,
                                 cudaStream_t stream) {
-  if (s.head_dim == 128)
-    return s.dual ? launch_one<128, true>(p, stream)
-                  : launch_one<128, false>(p, stream);
-  if (s.head_dim == 64)
-    return s.dual ? launch_one<64, true>(p, stream)
-                  : launch_one<64, false>(p, stream);
+  if (s.head_dim == 128) return launch_d<128>(p, s, stream);
+  if (s.head_dim == 64) return launch_d<64>(p, s, stream);
   return cudaErrorInvalidValue;
 }
 
 int attn_smem_bytes(const AttnLaunchShape& s) {
-  if (s.head_dim == 128)
-    return s.dual ? Cfg<128, true>::kSmem : Cfg<128, false>::kSmem;
-  if (s.head_dim == 64)
-    return s.dual ? Cfg<64, true>::kSmem : Cfg<64, false>::kSmem;
+  if (s.head_dim == 128) return smem_d<128>(s);
+  if (s.head_dim == 64) return smem_d<64>(s);
   return -1;
 }
 

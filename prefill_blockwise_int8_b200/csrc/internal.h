@@ -37,11 +37,13 @@ struct AttnParams {
   CUtensorMap tm_k;   // fp16 K  [T, hkv, d], box {64, 128, 1}
   CUtensorMap tm_k8;  // int8 K8 [T, hkv, d], box {d, 128, 1}
   CUtensorMap tm_v;   // fp16 V  [T, hkv, d], box {64, 128, 1}
+  CUtensorMap tm_v8;  // int8 V8 [T, hkv, d], box {d, 128, 1}, no swizzle
   const int32_t* cu_seqlens;
   const int32_t* head_map;
   const uint64_t* mask;
   const float* q_scale;
   const float* k_scale;
+  const float* v_scale;  // INT8 KV cache: [hkv, batch, nbk]
   uint16_t* out;     // fp16 bits [T, hq, d]
   float* lse;
   int32_t* qk_dump;
@@ -62,6 +64,7 @@ struct AttnParams {
 struct AttnLaunchShape {
   int head_dim;
   bool dual;  // routing rows of 64 inside 128-row compute tiles
+  bool kv8;   // K and V arrive as an INT8 cache (k8, v8 + block scales)
 };
 
 cudaError_t launch_attn_prefill(const AttnParams& p, const AttnLaunchShape& s,

@@ -191,9 +191,7 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
                 a->flags);
   if (a->kv_format != TILEMIX_KV_FP16 && a->kv_format != TILEMIX_KV_INT8)
     return fail(TILEMIX_ERR_INVALID_ARG, "attn: bad kv_format %d", a->kv_format);
-  if (a->kv_format == TILEMIX_KV_INT8)
-    return fail(TILEMIX_ERR_UNSUPPORTED,
-                "attn: the INT8 KV-cache format is not built yet");
+  const bool kv8 = a->kv_format == TILEMIX_KV_INT8;
   if (a->head_dim != 64 && a->head_dim != 128)
     return fail(TILEMIX_ERR_UNSUPPORTED, "attn: head_dim %d not in {64, 128}",
                 a->head_dim);
@@ -228,13 +226,20 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
     return fail(TILEMIX_ERR_INVALID_ARG,
                 "attn: ceil(%lld key tiles / g=%d) > 64 routing bits", tn,
                 a->group);
-  if (!a->q || !a->k || !a->v || !a->out || !a->cu_seqlens)
-    return fail(TILEMIX_ERR_INVALID_ARG, "attn: null q/k/v/out/cu_seqlens");
+  if (!a->q || !a->out || !a->cu_seqlens)
+    return fail(TILEMIX_ERR_INVALID_ARG, "attn: null q/out/cu_seqlens");
+  if (!kv8 && (!a->k || !a->v))
+    return fail(TILEMIX_ERR_INVALID_ARG, "attn: null k/v");
+  if (kv8 && (!a->k8 || !a->k_scale || !a->v8 || !a->v_scale))
+    return fail(TILEMIX_ERR_INVALID_ARG,
+                "attn: the INT8 KV cache needs k8, k_scale, v8 and v_scale");
   if (!fp16_only && (!a->mask || !a->q8 || !a->q_scale || !a->k8 || !a->k_scale))
     return fail(TILEMIX_ERR_INVALID_ARG,
                 "attn: mask, q8, q_scale, k8 and k_scale are required unless "
                 "TILEMIX_FLAG_FP16_ONLY is set");
-  if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) ||
+  if (!aligned(a->q, 16) || (a->k && !aligned(a->k, 16)) ||
+      (a->v && !aligned(a->v, 16)) || (a->v8 && !aligned(a->v8, 16)) ||
+      (a->v_scale && !aligned(a->v_scale, 4)) ||
       !aligned(a->out, 16) || !aligned(a->cu_seqlens, 4) ||
       (a->q8 && !aligned(a->q8, 16)) || (a->k8 && !aligned(a->k8, 16)) ||
       (a->q_scale && !aligned(a->q_scale, 4)) ||
@@ -260,23 +265,31 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   // The kernel computes 128 x 128 score tiles (a 64-key routing tile is one
   // half of a compute tile).
   bool maps = make_map(&p.tm_q, a->q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
-                       a->hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map(&p.tm_k, a->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
-                       a->hkv, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map(&p.tm_v, a->v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
-                       a->hkv, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+                       a->hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (maps && !kv8)
+    maps = make_map(&p.tm_k, a->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
+                    a->hkv, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+           make_map(&p.tm_v, a->v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
+                    a->hkv, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (maps && !fp16_only)
     maps = make_map(&p.tm_q8, a->q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
-                    a->hq, d, 128, i8sw) &&
-           make_map(&p.tm_k8, a->k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
+                    a->hq, d, 128, i8sw);
+  // The INT8 cache always feeds K8 (the INT8 path, or converted to fp16 on
+  // chip for FP16 groups) and V8 (converted to fp16 on chip).
+  if (maps && (kv8 || !fp16_only))
+    maps = make_map(&p.tm_k8, a->k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
                     a->hkv, d, 128, i8sw);
+  if (maps && kv8)
+    maps = make_map(&p.tm_v8, a->v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
+                    a->hkv, d, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!maps) return fail(TILEMIX_ERR_CUDA, "attn: tensor map encoding failed");
 
   p.cu_seqlens = a->cu_seqlens;
   p.head_map = a->head_map;
   p.mask = fp16_only ? nullptr : a->mask;
   p.q_scale = fp16_only ? nullptr : a->q_scale;
-  p.k_scale = fp16_only ? nullptr : a->k_scale;
+  p.k_scale = (fp16_only && !kv8) ? nullptr : a->k_scale;
+  p.v_scale = kv8 ? a->v_scale : nullptr;
   p.out = static_cast<uint16_t*>(a->out);
   p.lse = a->lse;
   p.qk_dump = a->qk_dump;
@@ -302,7 +315,7 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
       a->softmax_scale > 0.0f ? a->softmax_scale : 1.0f / std::sqrt(float(d));
   p.scale_log2 = scale * 1.4426950408889634f;
 
-  tilemix::AttnLaunchShape shape{d, a->block_m == 64};
+  tilemix::AttnLaunchShape shape{d, a->block_m == 64, kv8};
   cudaError_t e = tilemix::launch_attn_prefill(p, shape, stream);
   if (e != cudaSuccess)
     return fail(TILEMIX_ERR_CUDA, "attn launch: %s", cudaGetErrorString(e));

@@ -9,7 +9,9 @@ import workloads as W
 # fp64 oracle): max |gpu - ref| <= 3e-3 and ||gpu - ref||_2 / ||ref||_2 <=
 # 2e-3.  Error budget: half an fp16 ulp of the output (<= 9.8e-4 for
 # |o| < 4), fp16 rounding of P (relative 2^-11 per weight, <= 4.9e-4 * |v|),
-# ex2.approx (2 ulp) and fp32 score arithmetic (~1e-6 relative).
+# exp2 (ex2.approx 2 ulp; the FMA-pipe cubic 7.5e-5 relative), fp32 score
+# arithmetic (~1e-6 relative); with the INT8 KV cache, V = v8 * sv rounded to
+# fp16 on chip (relative 2^-10 per value).
 MAX_ABS = 3e-3
 REL_L2 = 2e-3
 LSE_ABS = 1e-3
@@ -42,6 +44,12 @@ def run_gpu(inp, *, fp16_only=False, want_lse=False, want_dump=False,
                                            status=status, stream=stream)
     k8, sk = tm.tilemix_quantize_blockwise(k, cu, ms, w.quant_block_k,
                                            status=status, stream=stream)
+    kv8 = w.kv_format == "int8"
+    v8 = sv = None
+    if kv8:  # the INT8 KV cache: K and V arrive quantised, fp16 K/V unused
+        v8, sv = tm.tilemix_quantize_blockwise(v, cu, ms, w.quant_block_k,
+                                               status=status, stream=stream)
+        k = v = None
     r = dev_tensor(inp["route"] if route is None else route)
     mask = tm.tilemix_pack_mask(r, cu, ms, w.block_m, w.block_n, g,
                                 status=status, stream=stream)
@@ -56,11 +64,12 @@ def run_gpu(inp, *, fp16_only=False, want_lse=False, want_dump=False,
     hm = dev_tensor(np.asarray(head_map, np.int32)) if head_map is not None \
         else None
     out = tm.tilemix_attn_prefill(
-        q, k, v, cu, ms, q8=q8, q_scale=sq, k8=k8, k_scale=sk, mask=mask,
-        block_m=w.block_m, block_n=w.block_n, group=g,
+        q, k, v, cu, ms, q8=q8, q_scale=sq, k8=k8, k_scale=sk, v8=v8,
+        v_scale=sv, mask=mask, block_m=w.block_m, block_n=w.block_n, group=g,
         quant_block_q=w.quant_block_q, quant_block_k=w.quant_block_k,
         head_map=hm, fp16_only=fp16_only, lse=lse, qk_dump=dump,
-        status=status, stream=stream)
+        kv_format=tm.KV_INT8 if kv8 else tm.KV_FP16, status=status,
+        stream=stream)
     torch.cuda.synchronize()
     res = dict(status=int(status.item()),
                out=out.float().cpu().numpy().astype(np.float64),

@@ -31,13 +31,13 @@ def tm():
 
 
 def small(L, *, hq=4, hkv=2, d=128, bm=128, bn=64, g=1, recipe="diag_first",
-          cov=0.75, seed=5, outliers=True, qb=128, kb=128):
+          cov=0.75, seed=5, outliers=True, qb=128, kb=128, kv="fp16"):
     lens = [L] if isinstance(L, int) else list(L)
     w = W.Workload(name="small", batch=len(lens), hq=hq, hkv=hkv, d=d,
                    block_m=bm, block_n=bn, group=g, seqlen=0, outliers=outliers,
                    mask_recipe=recipe, coverage=cov, seed=seed,
                    mask_seed=seed + 100, quant_block_q=qb, quant_block_k=kb,
-                   coverage_unit="kv_head")
+                   coverage_unit="kv_head", kv_format=kv)
     lens = np.array(lens, dtype=np.int32)
     # the fixed-length generator stream, drawn for T = sum(lens) tokens
     q, k, v = W.qkv(w.with_(seqlen=1), lens)
@@ -136,6 +136,13 @@ CASES = {
     "tiny_seqs_and_empty": ([1, 2, 0, 3, 130], dict(recipe="bernoulli", cov=0.5)),
     "exactly_64_groups": ([4096], dict(hq=2, hkv=1, recipe="exact", cov=0.5)),
     "exactly_64_groups_g2": ([8192], dict(hq=1, hkv=1, bn=64, g=2, recipe="exact", cov=0.5)),
+    # INT8 KV cache: K8 / V8 + block scales are the inputs
+    "kv8_d128_bn128": ([700, 129], dict(bn=128, kv="int8", recipe="exact", cov=0.5)),
+    "kv8_d128_bn64_kblock64": ([450], dict(kb=64, kv="int8", recipe="exact", cov=0.5)),
+    "kv8_d64_mha": ([333], dict(d=64, hq=3, hkv=3, bn=128, kv="int8", recipe="exact", cov=0.5)),
+    "kv8_dual": ([300], dict(bm=64, bn=64, kv="int8", recipe="bernoulli", cov=0.5)),
+    "kv8_all_int8": ([400], dict(kv="int8", recipe="exact", cov=1.0)),
+    "kv8_all_fp16": ([400], dict(kv="int8", recipe="exact", cov=0.0)),
 }
 
 
@@ -264,7 +271,15 @@ def test_head_map_out_of_range_sets_status(tm):
     assert status.item() == 5
 
 
-def test_int8_kv_format_reports_unsupported_until_built(tm):
+def test_int8_kv_cache_fp16_only_flag(tm):
+    inp = small([260], kv="int8", recipe="exact", cov=0.5)
+    got = run_gpu(inp, fp16_only=True)
+    assert got["status"] == 0
+    ref, _ = run_oracle(inp, fp16_only=True)
+    compare(got["out"], ref)
+
+
+def test_int8_kv_cache_needs_its_buffers(tm):
     inp = small([128])
     with pytest.raises(tm.TilemixError):
         tm.tilemix_attn_prefill(dev_tensor(inp["q"]), None, None,
@@ -278,8 +293,8 @@ def test_int8_kv_format_reports_unsupported_until_built(tm):
 # ----------------------------------------------------------------------------
 
 @pytest.mark.parametrize("wname", [
-    W.LLAMA32_3B_4K.name, W.VARLEN16.name, W.sweep_32k(75).name,
-    W.sweep_32k(0).name, W.sweep_32k(100).name])
+    W.LLAMA32_3B_4K.name, W.VARLEN16.name, W.INT8KV_16K.name,
+    W.sweep_32k(75).name, W.sweep_32k(0).name, W.sweep_32k(100).name])
 def test_full_size_sampled_rows(tm, wname):
     w = W.WORKLOADS[wname]
     inp = W.make(w)
