@@ -326,22 +326,42 @@ def run_gpu(args):
     out = torch.empty_like(q)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 4
+    # INT8 KV cache: K8, V8 and their scales are the inputs (quantised once,
+    # outside the timed region, by the same quantiser); a step quantises Q,
+    # packs the words and runs attention.
+    kv8 = w.kv_format == "int8"
+    v8 = sv = None
+    if kv8:
+        v8 = torch.empty((T, w.hkv, w.d), dtype=torch.int8, device=dev)
+        sv = torch.empty_like(sk)
+        tm.tilemix_quantize_blockwise(k, cu, ms, w.quant_block_k, x8=k8,
+                                      scale=sk, status=status)
+        tm.tilemix_quantize_blockwise(v, cu, ms, w.quant_block_k, x8=v8,
+                                      scale=sv, status=status)
+        torch.cuda.synchronize(dev)
+        t_h = {"q": t_h["q"], "route": t_h["route"], "k8": k8.cpu(),
+               "k_scale": sk.cpu(), "v8": v8.cpu(), "v_scale": sv.cpu()}
+        del k, v
+        k = v = None
+    launches_per_step = 3 if kv8 else 4
 
     def step(attn_events=None):
         tm.tilemix_quantize_blockwise(q, cu, ms, w.quant_block_q, x8=q8,
                                       scale=sq, status=status)
-        tm.tilemix_quantize_blockwise(k, cu, ms, w.quant_block_k, x8=k8,
-                                      scale=sk, status=status)
+        if not kv8:
+            tm.tilemix_quantize_blockwise(k, cu, ms, w.quant_block_k, x8=k8,
+                                          scale=sk, status=status)
         tm.tilemix_pack_mask(route, cu, ms, w.block_m, w.block_n, g, mask=mask,
                              status=status)
         if attn_events:
             attn_events[0].record(stream)
         tm.tilemix_attn_prefill(
-            q, k, v, cu, ms, q8=q8, q_scale=sq, k8=k8, k_scale=sk, mask=mask,
-            block_m=w.block_m, block_n=w.block_n, group=g,
-            quant_block_q=w.quant_block_q, quant_block_k=w.quant_block_k,
-            out=out, status=status)
+            q, k, v, cu, ms, q8=q8, q_scale=sq, k8=k8, k_scale=sk, v8=v8,
+            v_scale=sv, mask=mask, block_m=w.block_m, block_n=w.block_n,
+            group=g, quant_block_q=w.quant_block_q,
+            quant_block_k=w.quant_block_k,
+            kv_format=tm.KV_INT8 if kv8 else tm.KV_FP16, out=out,
+            status=status)
         if attn_events:
             attn_events[1].record(stream)
 
@@ -396,11 +416,15 @@ def run_gpu(args):
             cu_pin.numel() * 4
         d2h = out_h.numel() * out_h.element_size()
 
+        dev_of = {"q": q, "route": route}
+        if kv8:
+            dev_of.update(k8=k8, k_scale=sk, v8=v8, v_scale=sv)
+        else:
+            dev_of.update(k=k, v=v)
+
         def e2e_step():
-            q.copy_(pin["q"], non_blocking=True)
-            k.copy_(pin["k"], non_blocking=True)
-            v.copy_(pin["v"], non_blocking=True)
-            route.copy_(pin["route"], non_blocking=True)
+            for name, t in dev_of.items():
+                t.copy_(pin[name], non_blocking=True)
             cu.copy_(cu_pin, non_blocking=True)
             step()
             out_h.copy_(out, non_blocking=True)
