@@ -72,6 +72,18 @@ def measured_traffic(workload_name):
     return NCU_TRAFFIC.get((workload_name, kernel_source_hash()))
 
 
+def max_over_ranks(x: float, device) -> float:
+    """Largest value of x over all ranks of the default process group (x
+    itself without one): the job's time is its slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__,
                                  formatter_class=argparse.RawTextHelpFormatter)
@@ -84,6 +96,8 @@ def parse_args(argv=None):
                     choices=sorted(W.WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--ref-seconds", type=float, default=150.0,
+                    help="CPU time budget of the --impl reference run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args(argv)
@@ -165,7 +179,7 @@ def run_reference(args):
     import oracle
     oargs, kw = oracle.prepare(inp)
     total = int(inp["seqlens"].sum())
-    budget = 150.0  # seconds for warmup + steps together
+    budget = args.ref_seconds  # seconds for warmup + steps together
     per_step = budget / (args.steps + args.warmup)
     rng = np.random.default_rng(11)
     # calibrate rows per step
@@ -393,11 +407,7 @@ def run_gpu(args):
         dist.barrier()
     step_ms = [e[0].elapsed_time(e[3]) for e in ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    total_ms = sum(step_ms)
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()} in timed region")
     ms_step = total_ms / args.steps
@@ -440,11 +450,7 @@ def run_gpu(args):
             e2e_step()
             ee[i][1].record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = sum(a.elapsed_time(b) for a, b in ee)
-        if world > 1:
-            tt = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ee), dev)
         e2e = {"value": world * T / (e_ms / n_e2e * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": n_e2e}
