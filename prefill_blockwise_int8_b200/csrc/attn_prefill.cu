@@ -386,12 +386,12 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
     return r;
   };
   const TileRoute rt0 = route_of(0), rt1 = route_of(1);
-  auto rt = [&](int t) -> const TileRoute& { return t ? rt1 : rt0; };
+  auto rt = [&](int t) -> TileRoute { return t ? rt1 : rt0; };
   const int n_end = max(rt0.n_last, rt1.n_last);
   const int tpb = p.tiles_per_bit;  // 64-key blocks per routing bit
   // Paths query tile t needs for 64-key half kh of key tile n (0: none).
   auto kinds_of = [&](int t, int n, int kh) -> uint32_t {
-    const TileRoute& r = rt(t);
+    const TileRoute r = rt(t);
     const int n64 = 2 * n + kh;
     const int gi = n64 / tpb;
     uint32_t k = 0;
@@ -467,14 +467,25 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
   if (warp == kWarpProducer) {
     // =================== TMA producer ===================
     if (lane == 0) {
+      // Paths a query tile uses anywhere: its words' bits over the legal
+      // groups (bit set: INT8 somewhere; bit clear: FP16 somewhere).
+      auto need_of = [&](const TileRoute& r) -> uint32_t {
+        auto legal = [&](int nl) -> uint64_t {
+          if (nl < 0) return 0ull;
+          const int gl = nl / tpb;  // last legal group
+          return gl >= 63 ? ~0ull : ((1ull << (gl + 1)) - 1ull);
+        };
+        const uint64_t l0 = legal(r.nl0), l1 = legal(r.nl1);
+        uint32_t k = 0;
+        if ((r.w0 & l0) | (r.w1 & l1)) k |= kKindI8;
+        if ((~r.w0 & l0) | (~r.w1 & l1)) k |= kKindF16;
+        return k;
+      };
       uint32_t qbytes = 0;
-      uint32_t need[2] = {0u, 0u};
-      for (int t = 0; t < kQT; ++t) {
-        for (int n = 0; n <= rt(t).n_last; ++n)
-          need[t] |= kinds_of(t, n, 0) | kinds_of(t, n, 1);
+      const uint32_t need[2] = {need_of(rt0), need_of(rt1)};
+      for (int t = 0; t < kQT; ++t)
         qbytes += ((need[t] & kKindF16) ? C::kQBytes : 0) +
                   ((need[t] & kKindI8) ? C::kQ8Bytes : 0);
-      }
       mbar_arrive_expect_tx(&bars[C::kBarQ], qbytes);
       for (int t = 0; t < kQT; ++t) {
         const int qrow = start + row_base + t * kBM;
@@ -722,7 +733,7 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
     if (t < kQT) {
-      const TileRoute& R = rt(t);
+      const TileRoute R = rt(t);
       const int r_local = row_base + t * kBM + r;
       const int rh = DUAL ? (r >> 6) : 0;  // routing row half
       const uint64_t my_w = rh ? R.w1 : R.w0;
