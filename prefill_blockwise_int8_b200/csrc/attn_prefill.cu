@@ -121,7 +121,8 @@ struct Cfg {
   static constexpr int kBarO = kBarP + 2;              // [tile]
   static constexpr int kBarRed = kBarO + 2;            // [tile][parity]
   // INT8 KV cache: K slot holds its fp16 copy, V slot its fp16 V
-  static constexpr int kBarKConv = kBarRed + 4;        // [K slot]
+  static constexpr int kBarOStage = kBarRed + 4;       // [tile]
+  static constexpr int kBarKConv = kBarOStage + 2;     // [K slot]
   static constexpr int kBarVConv = kBarKConv + kKStages;  // [V slot]
   static constexpr int kBarDrain = kBarVConv + kVStages;
   static constexpr int kNumBars = kBarDrain + 1;
@@ -425,6 +426,7 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
       mbar_init(&bars[C::kBarS + i], 1);
       mbar_init(&bars[C::kBarP + i], 8);   // one arrival per softmax warp
       mbar_init(&bars[C::kBarO + i], 1);
+      mbar_init(&bars[C::kBarOStage + i], 8);  // O of tile i staged
       mbar_init(&bars[C::kBarRed + 2 * i], 8);
       mbar_init(&bars[C::kBarRed + 2 * i + 1], 8);
     }
@@ -438,6 +440,7 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_o);
     if (KV8) {
       tma_prefetch_desc(&p.tm_k8);
       tma_prefetch_desc(&p.tm_v8);
@@ -922,6 +925,11 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
             const bool valid = r_local < len;
             const float inv_l = 1.0f / l_tot;
             const int o0 = hw * (D / 2);
+            // A tile whose 128 rows all lie in the sequence leaves through
+            // one bulk store from shared memory (its Q buffer is free now);
+            // a partial tile stores its valid rows directly.
+            const bool full = row_base + t * kBM + kBM <= len;
+            uint8_t* stage = sQ(t);
             uint16_t* orow =
                 p.out + (static_cast<size_t>(start + r_local) * p.hq + h) * D +
                 o0;
@@ -935,12 +943,36 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
               for (int j = 0; j < 16; ++j)
                 hv[j] = pack_half2(__uint_as_float(o[2 * j]) * inv_l,
                                    __uint_as_float(o[2 * j + 1]) * inv_l);
-              if (valid) {
-                uint4* dst = reinterpret_cast<uint4*>(orow + oc);
 #pragma unroll
-                for (int v = 0; v < 4; ++v)
-                  dst[v] = make_uint4(hv[4 * v], hv[4 * v + 1], hv[4 * v + 2],
-                                      hv[4 * v + 3]);
+              for (int v = 0; v < 4; ++v) {
+                const uint4 val = make_uint4(hv[4 * v], hv[4 * v + 1],
+                                             hv[4 * v + 2], hv[4 * v + 3]);
+                if (full) {
+                  // column o0 + oc + 8v: chunk (o0 + oc) / 64, 16-byte
+                  // unit ((o0 + oc) % 64) / 8 + v of row r, 128B swizzle
+                  const int col = o0 + oc + 8 * v;
+                  const uint32_t off = (col / 64) * (kBM * 128) + r * 128 +
+                                       ((col % 64) / 8) * 16;
+                  *reinterpret_cast<uint4*>(stage + swz(off, 7)) = val;
+                } else if (valid) {
+                  reinterpret_cast<uint4*>(orow + oc)[v] = val;
+                }
+              }
+            }
+            if (full) {
+              fence_proxy_async_smem();  // staged O visible to the bulk copy
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars[C::kBarOStage + t]);
+              if (threadIdx.x == t * 256) {
+                if (mbar_wait(&bars[C::kBarOStage + t], 0, abort_flag)) {
+                  for (int c = 0; c < D / 64; ++c)
+                    tma_store_3d(&p.tm_o, stage + c * kBM * 128, c * 64,
+                                 start + row_base + t * kBM, h);
+                  bulk_commit_group();
+                  bulk_wait_all();
+                } else {
+                  ok = false;
+                }
               }
             }
             if (p.lse && valid && hw == 0)

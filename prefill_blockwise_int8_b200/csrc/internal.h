@@ -38,6 +38,7 @@ struct AttnParams {
   CUtensorMap tm_k8;  // int8 K8 [T, hkv, d], box {d, 128, 1}
   CUtensorMap tm_v;   // fp16 V  [T, hkv, d], box {64, 128, 1}
   CUtensorMap tm_v8;  // int8 V8 [T, hkv, d], box {d, 128, 1}, no swizzle
+  CUtensorMap tm_o;   // fp16 O  [T, hq, d], box {64, 128, 1}, 128B swizzle
   const int32_t* cu_seqlens;
   const int32_t* head_map;
   const uint64_t* mask;

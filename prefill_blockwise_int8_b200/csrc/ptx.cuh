@@ -118,6 +118,29 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m,
       : "memory");
 }
 
+// 3-D tiled bulk store shared -> global (no multicast): the box at
+// coordinates {c0, c1, c2} of the map's tensor from `src`, in this thread's
+// bulk async-group.  c0 * element size must be a multiple of 16 bytes and
+// no coordinate may be negative.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m,
+                                             const void* src, int c0, int c1,
+                                             int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, "
+      "%4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until every bulk store this thread committed has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05: TMEM allocation
 // ---------------------------------------------------------------------------

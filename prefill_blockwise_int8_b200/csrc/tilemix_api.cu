@@ -265,7 +265,9 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   // The kernel computes 128 x 128 score tiles (a 64-key routing tile is one
   // half of a compute tile).
   bool maps = make_map(&p.tm_q, a->q, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
-                       a->hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+                       a->hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&p.tm_o, a->out, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d,
+                       T, a->hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (maps && !kv8)
     maps = make_map(&p.tm_k, a->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
                     a->hkv, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
