@@ -189,31 +189,6 @@ __device__ __forceinline__ float max64(const uint32_t (&sv)[64], int hl) {
   }
 }
 
-// 2^x of a pair on the FMA and integer pipes, for the share of the
-// exponentials taken off the MUFU: x = j + f with j the nearest integer and
-// |f| <= 1/2; 2^f from a cubic fitted to 2^f on [-1/2, 1/2] by Remez
-// exchange (relative error <= 7.5e-5, below the fp16 rounding of P); 2^j
-// added to the exponent bits.  x is clamped to >= -125 so the result stays
-// normal (2^-125 stands for 0: it vanishes in fp16 and in the fp32 sums).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f,
-                  kC3 = 0.055171669f;
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
-  const float2 t = __fadd2_rn(x, make_float2(kIntBias, kIntBias));
-  const float2 j = __fadd2_rn(t, make_float2(-kIntBias, -kIntBias));
-  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
-  float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-  q = __ffma2_rn(q, f, make_float2(kC1, kC1));
-  q = __ffma2_rn(q, f, make_float2(kC0, kC0));
-  return make_float2(
-      __uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-      __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
-}
-
-// Pairs of each 16-pair group computed by exp2_poly2 instead of the MUFU.
-constexpr int kPolyEvery = 4;
-
 // P = 2^(S c - m) of 32 scores as 16 packed fp16 pairs (key 2i in the low
 // half of pk[i]), added to four packed partial sums.  INT32 accumulators
 // convert to fp32 exactly (|acc| <= 127^2 d < 2^22) by the bias trick, on
@@ -246,9 +221,7 @@ __device__ __forceinline__ void exp32(const uint32_t (&sv)[32], float c,
       if (i & 1) xb = fmax3(xb, x.x, x.y);
       else xa = fmax3(xa, x.x, x.y);
     }
-    const float2 pr = (i % kPolyEvery == kPolyEvery - 1)
-                          ? exp2_poly2(x)
-                          : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
     switch (i & 3) {
       case 0: ps0 = __fadd2_rn(ps0, pr); break;
       case 1: ps1 = __fadd2_rn(ps1, pr); break;
