@@ -1,0 +1,86 @@
+"""Numerical-deviation study: how far tile-routed FP16/INT8 attention moves
+from the all-FP16 result as INT8 coverage grows.
+
+The TileMix paperlayer summary, appendix G Numerical Analysis (G.1, G.3),
+measures MaxDiff / MeanDiff of the routed kernel against a fixed FP16
+reference across INT8 coverage and precision layouts.  Here the fixed
+reference is this library's own FP16 path (TILEMIX_FLAG_FP16_ONLY: every
+legal tile FP16, same kernel, same schedule), so a difference isolates what
+INT8 routing changes.  Inputs are synthetic (seeded N(0,1) with outlier
+channels in Q and K, the same generator as the benchmark); routing masks
+draw exactly round(c * N_legal) INT8 groups per KV head.
+
+    python -m prefill_blockwise_int8_b200.deviation --seqlen 8192
+
+Needs a GPU; prints one line per coverage and returns the rows.
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import sys
+
+import numpy as np
+
+DEFAULT_COVERAGES = (0.0, 0.05, 0.10, 0.25, 0.50, 0.75, 1.0)
+
+
+def run(seqlen: int = 8192, hq: int = 8, hkv: int = 2, d: int = 128,
+        block_m: int = 128, block_n: int = 128, coverages=DEFAULT_COVERAGES,
+        seed: int = 7, device: str = "cuda"):
+    import torch
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    if root not in sys.path:
+        sys.path.insert(0, root)
+    import workloads as W
+    import prefill_blockwise_int8_b200 as tm
+
+    base = W.Workload(name="deviation", batch=1, hq=hq, hkv=hkv, d=d,
+                      block_m=block_m, block_n=block_n, group=0,
+                      seqlen=seqlen, outliers=True, mask_recipe="exact",
+                      coverage=0.0, coverage_unit="kv_head", seed=seed,
+                      mask_seed=seed + 1)
+    inp = W.make(base)
+    dev = torch.device(device)
+    cu = torch.from_numpy(inp["cu_seqlens"]).to(dev)
+    q, k, v = (torch.from_numpy(inp[x]).to(dev) for x in "qkv")
+    ms, g = inp["max_seqlen"], inp["group"]
+    q8, sq = tm.tilemix_quantize_blockwise(q, cu, ms, 128)
+    k8, sk = tm.tilemix_quantize_blockwise(k, cu, ms, 128)
+    ref = tm.tilemix_attn_prefill(q, k, v, cu, ms, fp16_only=True,
+                                  block_m=block_m, block_n=block_n,
+                                  group=g).float()
+    rows = []
+    for c in coverages:
+        w = base.with_(coverage=float(c), mask_seed=seed + 1 + int(c * 1000))
+        route = torch.from_numpy(W.route_bytes(w, inp["seqlens"])).to(dev)
+        mask = tm.tilemix_pack_mask(route, cu, ms, block_m, block_n, g)
+        out = tm.tilemix_attn_prefill(
+            q, k, v, cu, ms, q8=q8, q_scale=sq, k8=k8, k_scale=sk, mask=mask,
+            block_m=block_m, block_n=block_n, group=g).float()
+        diff = (out - ref).abs()
+        rows.append(dict(coverage=float(c), max_diff=float(diff.max()),
+                         mean_diff=float(diff.mean())))
+    return rows
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--seqlen", type=int, default=8192)
+    ap.add_argument("--hq", type=int, default=8)
+    ap.add_argument("--hkv", type=int, default=2)
+    ap.add_argument("--block-n", type=int, default=128)
+    args = ap.parse_args(argv)
+    rows = run(seqlen=args.seqlen, hq=args.hq, hkv=args.hkv,
+               block_n=args.block_n)
+    print(f"{'INT8 coverage':>14} {'MaxDiff':>10} {'MeanDiff':>10}")
+    for r in rows:
+        print(f"{r['coverage']:>14.2f} {r['max_diff']:>10.3e} "
+              f"{r['mean_diff']:>10.3e}")
+    return rows
+
+
+if __name__ == "__main__":
+    main()
