@@ -119,6 +119,56 @@ tilemix_status tilemix_pack_mask(
     uint64_t* mask, int32_t* status, tilemix_stream_t stream);
 
 /*
+ * Static routing templates: route bytes (1 = INT8, 0 = FP16) for a named
+ * spatial layout at a given INT8 coverage, ready for tilemix_pack_mask.
+ * Pages: paperlayer summary appendix B Precision Layouts (uniform All INT8
+ * and All FP16 references; Band, Global, Row-Random, Aligned Sparse,
+ * BigBird and SpTrans templates; 25/50/75% = INT8 share of legal tile
+ * groups) and Limitations (static templates give deterministic policies;
+ * the kernel consumes any static or adaptive policy).  The pages give the
+ * names only; the definitions below are this library's readings.
+ *
+ * Per query-tile row (b, hk, m) with G legal groups (the groups holding a
+ * causal in-sequence pair; group j covers key tiles g*j .. g*j+g-1) and
+ * distance d = G - 1 - j from the diagonal group:
+ *   k_int8 = (int8_permille * G + 500) / 1000 (integer division),
+ *   FP16 goes to the G - k_int8 groups with the largest key
+ *   (priority(j) << 32) | h32(j), ties to the smaller j, where h32 is the
+ *   high half of splitmix64 (Steele, Lea and Flood 2014) of
+ *   seed + (c + 1) * 0x9E3779B97F4A7C15 with counter
+ *   c = ((b * hkv + hk) * Tm_max + m) * 64 + j:
+ *     ALL_FP16     every legal group FP16 (int8_permille ignored)
+ *     ALL_INT8     every legal group INT8 (int8_permille ignored)
+ *     BAND         priority 63 - d     (FP16 band along the diagonal)
+ *     GLOBAL       priority 63 - j     (FP16 on the first key groups)
+ *     ROW_RANDOM   priority 0          (a random subset of each row)
+ *     ALIGNED      priority 1 when j % 4 == 0, else 0
+ *     BIGBIRD      priority 1 when j == 0 or d <= 1, else 0
+ *     SPTRANS      priority 2 when d <= 1, 1 when j % 4 == 3, else 0
+ * Bytes of illegal groups and of rows past a sequence are 0.
+ *
+ *   layout         TILEMIX_LAYOUT_*
+ *   int8_permille  INT8 share of each row's legal groups, in [0, 1000]
+ *   route          dev uint8 [batch, hkv, Tm_max, 64] (written entirely)
+ *   other arguments as for tilemix_pack_mask
+ */
+enum {
+  TILEMIX_LAYOUT_ALL_FP16 = 0,
+  TILEMIX_LAYOUT_ALL_INT8 = 1,
+  TILEMIX_LAYOUT_BAND = 2,
+  TILEMIX_LAYOUT_GLOBAL = 3,
+  TILEMIX_LAYOUT_ROW_RANDOM = 4,
+  TILEMIX_LAYOUT_ALIGNED = 5,
+  TILEMIX_LAYOUT_BIGBIRD = 6,
+  TILEMIX_LAYOUT_SPTRANS = 7
+};
+
+tilemix_status tilemix_route_template(
+    int layout, int int8_permille, uint64_t seed, const int32_t* cu_seqlens,
+    int batch, int max_seqlen, int hkv, int block_m, int block_n, int group,
+    uint8_t* route, int32_t* status, tilemix_stream_t stream);
+
+/*
  * Arguments of tilemix_attn_prefill.  Zero-initialise, set struct_size =
  * sizeof(tilemix_attn_params), then fill the fields.
  */

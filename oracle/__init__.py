@@ -240,3 +240,73 @@ def prepare(inputs: dict, fp16_only: bool = False):
     else:
         args = (cu, ms, inputs["q"], inputs["k"], inputs["v"])
     return args, kw
+
+
+# ----------------------------------------------------------------------------
+# Static routing templates (paperlayer summary, appendix B Precision Layouts:
+# All FP16 / All INT8 references, Band, Global, Row-Random, Aligned Sparse,
+# BigBird and SpTrans at an INT8 coverage of the legal tile groups).  The
+# pages give the names only; this restates the reading documented with the
+# C declaration of tilemix_route_template: per query-tile row, the
+# G - round(c G) groups with the highest (priority, hash) key stay FP16.
+# ----------------------------------------------------------------------------
+
+LAYOUTS = {"all_fp16": 0, "all_int8": 1, "band": 2, "global": 3,
+           "row_random": 4, "aligned": 5, "bigbird": 6, "sptrans": 7}
+_M64 = (1 << 64) - 1
+
+
+def splitmix64(z: int) -> int:
+    """The output function of the splitmix64 generator (Steele, Lea and
+    Flood, OOPSLA 2014): two xor-shift-multiply rounds and a final xor."""
+    z &= _M64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _M64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _M64
+    return z ^ (z >> 31)
+
+
+def _priority(layout: int, j: int, d: int) -> int:
+    if layout == LAYOUTS["band"]:
+        return 63 - d
+    if layout == LAYOUTS["global"]:
+        return 63 - j
+    if layout == LAYOUTS["aligned"]:
+        return 1 if j % 4 == 0 else 0
+    if layout == LAYOUTS["bigbird"]:
+        return 1 if (j == 0 or d <= 1) else 0
+    if layout == LAYOUTS["sptrans"]:
+        return 2 if d <= 1 else (1 if j % 4 == 3 else 0)
+    return 0
+
+
+def route_template(layout, int8_permille: int, seed: int, cu_seqlens,
+                   max_seqlen: int, hkv: int, block_m: int, block_n: int,
+                   group: int) -> np.ndarray:
+    """uint8 [batch, hkv, ceil(max_seqlen / block_m), 64], 1 = INT8."""
+    code = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    lens = np.diff(cu)
+    tm = -(-max_seqlen // block_m)
+    out = np.zeros((len(lens), hkv, tm, 64), dtype=np.uint8)
+    for b, L in enumerate(lens.tolist()):
+        for m in range(tm):
+            if m * block_m >= L:
+                continue
+            G = ((min((m + 1) * block_m, L) - 1) // block_n) // group + 1
+            k_int8 = (int8_permille * G + 500) // 1000
+            if code == LAYOUTS["all_fp16"]:
+                k_int8 = 0
+            if code == LAYOUTS["all_int8"]:
+                k_int8 = G
+            k_fp16 = G - k_int8
+            for hk in range(hkv):
+                keys = []
+                for j in range(G):
+                    c = ((b * hkv + hk) * tm + m) * 64 + j
+                    h = splitmix64(seed + (c + 1) * 0x9E3779B97F4A7C15) >> 32
+                    keys.append((_priority(code, j, G - 1 - j) << 32) | h)
+                # FP16: the k_fp16 largest keys, ties to the smaller index
+                order = sorted(range(G), key=lambda i: (-keys[i], i))
+                for j in order[k_fp16:]:
+                    out[b, hk, m, j] = 1
+    return out

@@ -24,8 +24,9 @@ from pathlib import Path
 __all__ = [
     "TilemixError", "lib", "library_path", "EXPORTED_SYMBOLS",
     "tilemix_quantize_blockwise", "tilemix_pack_mask", "tilemix_attn_prefill",
-    "tilemix_status_string", "tilemix_last_error", "tilemix_version",
-    "KV_FP16", "KV_INT8", "FLAG_FP16_ONLY", "STATUS",
+    "tilemix_route_template", "tilemix_status_string", "tilemix_last_error",
+    "tilemix_version", "KV_FP16", "KV_INT8", "FLAG_FP16_ONLY", "STATUS",
+    "LAYOUTS",
 ]
 
 _LIB_PATH = Path(__file__).resolve().parent / "libtilemix.so"
@@ -37,10 +38,15 @@ STATUS = {0: "TILEMIX_OK", 1: "TILEMIX_ERR_INVALID_ARG",
           4: "TILEMIX_ERR_TIMEOUT", 5: "TILEMIX_ERR_BAD_SEQLENS",
           6: "TILEMIX_ERR_NO_DEVICE"}
 
+# Routing-template layouts (TILEMIX_LAYOUT_*).
+LAYOUTS = {"all_fp16": 0, "all_int8": 1, "band": 2, "global": 3,
+           "row_random": 4, "aligned": 5, "bigbird": 6, "sptrans": 7}
+
 # Every function include/tilemix.h declares.
 EXPORTED_SYMBOLS = (
     "tilemix_quantize_blockwise", "tilemix_pack_mask", "tilemix_attn_prefill",
-    "tilemix_status_string", "tilemix_last_error", "tilemix_version",
+    "tilemix_route_template", "tilemix_status_string", "tilemix_last_error",
+    "tilemix_version",
 )
 
 
@@ -88,6 +94,9 @@ def _load() -> C.CDLL:
     lib.tilemix_pack_mask.restype = i32
     lib.tilemix_pack_mask.argtypes = [
         vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+    lib.tilemix_route_template.restype = i32
+    lib.tilemix_route_template.argtypes = [
+        i32, i32, C.c_uint64, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
     lib.tilemix_attn_prefill.restype = i32
     lib.tilemix_attn_prefill.argtypes = [C.POINTER(AttnParams), vp]
     lib.tilemix_status_string.restype = C.c_char_p
@@ -99,7 +108,29 @@ def _load() -> C.CDLL:
     return lib
 
 
-lib = _load()
+class _Missing:
+    """Stands in for the library when it is missing or older than the
+    sources (so the package imports for a build); any use raises."""
+
+    def __init__(self, err: Exception):
+        self._err = err
+
+    def __getattr__(self, name):
+        raise ImportError(f"libtilemix.so unusable ({self._err}); build it "
+                          "with `python -m prefill_blockwise_int8_b200.build`")
+
+
+try:
+    lib = _load()
+except (OSError, AttributeError, ImportError) as _e:
+    lib = _Missing(_e)
+
+
+def reload_library():
+    """Load libtilemix.so again (after a build)."""
+    global lib
+    lib = _load()
+    return lib
 
 
 def tilemix_status_string(status: int) -> str:
@@ -198,6 +229,29 @@ def tilemix_pack_mask(route, cu_seqlens, max_seqlen: int, block_m: int,
         block_n, group, _ptr(mask), _ptr(status), _stream(stream)),
         "tilemix_pack_mask")
     return mask
+
+
+def tilemix_route_template(layout, int8_permille: int, cu_seqlens,
+                           max_seqlen: int, hkv: int, block_m: int,
+                           block_n: int, group: int, *, seed: int = 0,
+                           route=None, status=None, stream=None):
+    """Route bytes [B, Hkv, ceil(max_seqlen/block_m), 64] (uint8, 1 = INT8)
+    of a named layout ("band", "bigbird", ... or a TILEMIX_LAYOUT_* value)
+    with an INT8 share of int8_permille / 1000 of each row's legal groups."""
+    torch = _torch()
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    code = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    batch = cu_seqlens.numel() - 1
+    tm = -(-max_seqlen // block_m)
+    if route is None:
+        route = torch.empty((batch, hkv, tm, 64), dtype=torch.uint8,
+                            device=cu_seqlens.device)
+    _dev(route, "route", torch.uint8)
+    _check(lib.tilemix_route_template(
+        code, int8_permille, seed & 0xFFFFFFFFFFFFFFFF, _ptr(cu_seqlens), batch,
+        max_seqlen, hkv, block_m, block_n, group, _ptr(route), _ptr(status),
+        _stream(stream)), "tilemix_route_template")
+    return route
 
 
 def tilemix_attn_prefill(q, k, v, cu_seqlens, max_seqlen: int, *, q8=None,

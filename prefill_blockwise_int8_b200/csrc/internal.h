@@ -29,6 +29,17 @@ cudaError_t launch_pack_mask(const uint8_t* route, const int32_t* cu_seqlens,
                              int block_n, int group, uint64_t* mask,
                              int32_t* status, cudaStream_t stream);
 
+// Routing-template layouts (same values as TILEMIX_LAYOUT_*).
+constexpr int kLayoutAllFp16 = 0, kLayoutAllInt8 = 1, kLayoutBand = 2,
+              kLayoutGlobal = 3, kLayoutRowRandom = 4, kLayoutAligned = 5,
+              kLayoutBigBird = 6, kLayoutSpTrans = 7;
+
+cudaError_t launch_route_template(int layout, int permille, uint64_t seed,
+                                  const int32_t* cu_seqlens, int batch,
+                                  int max_seqlen, int hkv, int block_m,
+                                  int block_n, int group, uint8_t* route,
+                                  int32_t* status, cudaStream_t stream);
+
 // Everything the fused attention kernel reads.  Passed by value as a
 // __grid_constant__ parameter; the tensor maps must stay 64-byte aligned.
 struct AttnParams {

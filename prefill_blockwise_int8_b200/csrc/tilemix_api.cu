@@ -176,6 +176,44 @@ tilemix_status tilemix_pack_mask(const uint8_t* route,
   return ok();
 }
 
+tilemix_status tilemix_route_template(int layout, int int8_permille,
+                                      uint64_t seed, const int32_t* cu_seqlens,
+                                      int batch, int max_seqlen, int hkv,
+                                      int block_m, int block_n, int group,
+                                      uint8_t* route, int32_t* status,
+                                      tilemix_stream_t stream) {
+  if (!route || !cu_seqlens)
+    return fail(TILEMIX_ERR_INVALID_ARG, "route_template: null pointer");
+  if (!aligned(route, 16) || !aligned(cu_seqlens, 4) ||
+      (status && !aligned(status, 4)))
+    return fail(TILEMIX_ERR_INVALID_ARG, "route_template: misaligned pointer");
+  if (layout < TILEMIX_LAYOUT_ALL_FP16 || layout > TILEMIX_LAYOUT_SPTRANS)
+    return fail(TILEMIX_ERR_INVALID_ARG, "route_template: bad layout %d",
+                layout);
+  if (int8_permille < 0 || int8_permille > 1000)
+    return fail(TILEMIX_ERR_INVALID_ARG,
+                "route_template: int8_permille %d not in [0, 1000]",
+                int8_permille);
+  if (batch < 0 || max_seqlen < 0 || hkv <= 0 || block_m <= 0 ||
+      block_n <= 0 || group <= 0)
+    return fail(TILEMIX_ERR_INVALID_ARG, "route_template: bad size");
+  if (batch == 0 || max_seqlen == 0) return ok();
+  const long long tn = (static_cast<long long>(max_seqlen) + block_n - 1) / block_n;
+  if ((tn + group - 1) / group > 64)
+    return fail(TILEMIX_ERR_INVALID_ARG,
+                "route_template: ceil(%lld key tiles / g=%d) > 64 routing bits",
+                tn, group);
+  tilemix_status d = check_device();
+  if (d != TILEMIX_OK) return d;
+  cudaError_t e = tilemix::launch_route_template(
+      layout, int8_permille, seed, cu_seqlens, batch, max_seqlen, hkv, block_m,
+      block_n, group, route, status, stream);
+  if (e != cudaSuccess)
+    return fail(TILEMIX_ERR_CUDA, "route_template launch: %s",
+                cudaGetErrorString(e));
+  return ok();
+}
+
 tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
                                     tilemix_stream_t stream) {
   if (!a) return fail(TILEMIX_ERR_INVALID_ARG, "attn: params is NULL");

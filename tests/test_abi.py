@@ -140,3 +140,17 @@ def test_quantize_and_pack_host_checks():
     assert pk(FAKE, FAKE, 1, 64 * 65, 1, 64, 64, 2, FAKE, None, None) in (NO_DEVICE, OK)
     assert pk(FAKE + 8, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
     assert pk(None, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
+
+
+def test_route_template_host_checks():
+    rt = tm.lib.tilemix_route_template
+    # layout, int8_permille, seed, cu, batch, max_seqlen, hkv, bm, bn, g, route
+    assert rt(2, 750, 1, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) in (NO_DEVICE, OK)
+    assert rt(8, 750, 1, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
+    assert rt(-1, 750, 1, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
+    assert rt(2, 1001, 1, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
+    assert rt(2, -1, 1, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
+    assert rt(2, 750, 1, FAKE, 1, 64 * 65, 1, 64, 64, 1, FAKE, None, None) == INVALID
+    assert rt(2, 750, 1, FAKE, 1, 128, 1, 64, 64, 1, FAKE + 8, None, None) == INVALID
+    assert rt(2, 750, 1, None, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
+    assert rt(2, 750, 1, FAKE, 0, 0, 1, 64, 64, 1, FAKE, None, None) == OK

@@ -307,3 +307,38 @@ def test_full_size_sampled_rows(tm, wname):
     assert np.array_equal(got["sq"].view(np.uint32), kw["q_scale"].view(np.uint32))
     assert np.array_equal(got["mask"], kw["mask"])
     compare(got["out"], ref, rows=rows)
+
+
+# ----------------------------------------------------------------------------
+# routing templates: byte-exact against the oracle, then through attention
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("layout", sorted(oracle.LAYOUTS))
+def test_route_template_bitexact(tm, layout):
+    shapes = [([700, 300, 1, 0, 1500], 2, 128, 64, 1),
+              ([4096] * 8, 8, 128, 64, 1),
+              ([8192], 2, 128, 128, 1),
+              ([20000], 1, 64, 64, 5)]
+    for lens, hkv, bm, bn, g in shapes:
+        lens = np.array(lens, np.int32)
+        cu = W.cu_seqlens(lens)
+        ms = int(max(lens.max(), 1))
+        for permille in (0, 250, 500, 750, 1000):
+            got = tm.tilemix_route_template(layout, permille, dev_tensor(cu),
+                                            ms, hkv, bm, bn, g, seed=77)
+            torch.cuda.synchronize()
+            ref = oracle.route_template(layout, permille, 77, cu, ms, hkv, bm,
+                                        bn, g)
+            assert np.array_equal(got.cpu().numpy(), ref), (lens, permille)
+
+
+def test_route_template_through_attention(tm):
+    inp = small([900, 333], bn=64)
+    w = inp["workload"]
+    route = tm.tilemix_route_template(
+        "bigbird", 750, dev_tensor(inp["cu_seqlens"]), inp["max_seqlen"],
+        w.hkv, w.block_m, w.block_n, inp["group"], seed=5).cpu().numpy()
+    got = run_gpu(inp, route=route)
+    assert got["status"] == 0
+    ref, _ = run_oracle(inp, route=route)
+    compare(got["out"], ref)

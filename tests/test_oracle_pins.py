@@ -405,3 +405,65 @@ def test_qk_dump_equals_integer_matmul():
                 else:
                     assert (tile == -1).all()
     assert seen > 0
+
+
+# ----------------------------------------------------------------------------
+# routing templates: coverage per row, structure of each layout
+# ----------------------------------------------------------------------------
+
+def _legal_groups(L, m, bm, bn, g):
+    return ((min((m + 1) * bm, L) - 1) // bn) // g + 1 if m * bm < L else 0
+
+
+@pytest.mark.parametrize("layout", sorted(oracle.LAYOUTS))
+@pytest.mark.parametrize("permille", [0, 250, 500, 750, 1000])
+def test_route_template_coverage_and_legality(layout, permille):
+    cu = np.array([0, 700, 1000, 1001], np.int64)
+    bm, bn, g, hkv = 128, 64, 1, 2
+    r = oracle.route_template(layout, permille, 3, cu, 700, hkv, bm, bn, g)
+    for b, L in enumerate(np.diff(cu)):
+        for m in range(r.shape[2]):
+            G = _legal_groups(int(L), m, bm, bn, g)
+            row = r[b, :, m, :]
+            assert (row[:, G:] == 0).all()  # illegal groups and empty rows
+            if G == 0:
+                continue
+            k8 = {"all_fp16": 0, "all_int8": G}.get(
+                layout, (permille * G + 500) // 1000)
+            assert (row[:, :G].sum(axis=1) == k8).all()
+
+
+def test_route_template_structure():
+    cu = np.array([0, 2048], np.int64)
+    G = 2048 // 64  # last query-tile row: 32 legal groups
+    def last_row(layout, permille):
+        return oracle.route_template(layout, permille, 9, cu, 2048, 1, 128,
+                                     64, 1)[0, 0, 15, :G]
+    fp16 = lambda row: set(np.nonzero(row == 0)[0].tolist())
+    # band: FP16 are the groups nearest the diagonal; global: the first ones
+    assert fp16(last_row("band", 750)) == set(range(G - 8, G))
+    assert fp16(last_row("global", 750)) == set(range(8))
+    # bigbird: group 0 and the two diagonal groups come first
+    assert {0, G - 2, G - 1} <= fp16(last_row("bigbird", 750))
+    assert fp16(last_row("bigbird", 1000 - 94)) == {0, G - 2, G - 1}
+    # sptrans: local pair first, then every fourth group (j % 4 == 3)
+    assert fp16(last_row("sptrans", 1000 - 63)) == {G - 2, G - 1}
+    strided = {j for j in range(G) if j % 4 == 3}
+    assert fp16(last_row("sptrans", 500)) >= {G - 2, G - 1}
+    assert fp16(last_row("sptrans", 500)) <= strided | {G - 2, G - 1} | set(range(G))
+    sp = fp16(last_row("sptrans", 750))  # 8 FP16: local 2 + 6 strided
+    assert {G - 2, G - 1} <= sp and len(sp - {G - 2, G - 1} - strided) == 0
+    # aligned: FP16 on j % 4 == 0 first
+    al = fp16(last_row("aligned", 750))
+    assert al <= {j for j in range(G) if j % 4 == 0}
+    # row-random: exact count, depends on the seed and on the row
+    a = oracle.route_template("row_random", 500, 1, cu, 2048, 2, 128, 64, 1)
+    b = oracle.route_template("row_random", 500, 2, cu, 2048, 2, 128, 64, 1)
+    assert not np.array_equal(a, b)
+    assert not np.array_equal(a[0, 0], a[0, 1])
+
+
+def test_splitmix64_is_a_bijection_on_a_sample():
+    vals = {oracle.splitmix64(x) for x in range(1 << 14)}
+    assert len(vals) == 1 << 14
+    assert all(0 <= v < (1 << 64) for v in vals)
