@@ -98,6 +98,9 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
                     help="CPU time budget of the --impl reference run")
+    ap.add_argument("--quant-on-chip", action="store_true",
+                    help="quantise Q and K tiles inside the attention kernel "
+                         "(no separate quantiser launches)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args(argv)
@@ -357,12 +360,14 @@ def run_gpu(args):
                "k_scale": sk.cpu(), "v8": v8.cpu(), "v_scale": sv.cpu()}
         del k, v
         k = v = None
-    launches_per_step = 3 if kv8 else 4
+    on_chip = args.quant_on_chip and not kv8
+    launches_per_step = 2 if on_chip else (3 if kv8 else 4)
 
     def step(attn_events=None):
-        tm.tilemix_quantize_blockwise(q, cu, ms, w.quant_block_q, x8=q8,
-                                      scale=sq, status=status)
-        if not kv8:
+        if not on_chip:
+            tm.tilemix_quantize_blockwise(q, cu, ms, w.quant_block_q, x8=q8,
+                                          scale=sq, status=status)
+        if not kv8 and not on_chip:
             tm.tilemix_quantize_blockwise(k, cu, ms, w.quant_block_k, x8=k8,
                                           scale=sk, status=status)
         tm.tilemix_pack_mask(route, cu, ms, w.block_m, w.block_n, g, mask=mask,
@@ -374,8 +379,8 @@ def run_gpu(args):
             v_scale=sv, mask=mask, block_m=w.block_m, block_n=w.block_n,
             group=g, quant_block_q=w.quant_block_q,
             quant_block_k=w.quant_block_k,
-            kv_format=tm.KV_INT8 if kv8 else tm.KV_FP16, out=out,
-            status=status)
+            kv_format=tm.KV_INT8 if kv8 else tm.KV_FP16,
+            quant_on_chip=on_chip, out=out, status=status)
         if attn_events:
             attn_events[1].record(stream)
 
@@ -496,7 +501,8 @@ def run_gpu(args):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp16+int8", "data": "synthetic",
-        "config": workload_config(w, inp, wk["int8_pair_share"]),
+        "config": dict(workload_config(w, inp, wk["int8_pair_share"]),
+                       quantisation="on chip" if on_chip else "quantise once"),
         "effective_tflops": wk["effective"] / (ms_step * 1e-3) / 1e12 * world,
         "attn_effective_tflops": achieved,
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,

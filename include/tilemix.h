@@ -67,6 +67,16 @@ enum { TILEMIX_KV_FP16 = 0, TILEMIX_KV_INT8 = 1 };
  * NULL.  This is the all-FP16 reference mode. */
 #define TILEMIX_FLAG_FP16_ONLY 1u
 
+/* On-the-fly quantisation (paperlayer summary, appendix C Quantization
+ * Configuration: INT8 fragments generated only for routed groups, scales
+ * computed and applied on chip).  The kernel quantises each Q tile and each
+ * key tile that some row routes to INT8 itself, with the quantiser's exact
+ * definition (one scale per 128-token block; needs quant_block_q =
+ * quant_block_k = 128), so results equal a tilemix_quantize_blockwise call
+ * followed by the quantize-once attention.  q8, q_scale, k8 and k_scale are
+ * not read (may be NULL).  TILEMIX_KV_FP16 only. */
+#define TILEMIX_FLAG_QUANT_ON_CHIP 2u
+
 /*
  * Blockwise symmetric INT8 quantisation ("quantize-once").
  * Pages: section 3 Preliminaries (blockwise quantization; INT8 tensor cores

@@ -38,6 +38,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "quant_code.cuh"
 
 namespace tilemix {
 namespace {
@@ -47,9 +48,15 @@ constexpr int kBN = 128;     // keys per compute tile
 constexpr int kHalf = 64;    // routing granularity inside a compute tile
 constexpr int kWarpProducer = 16;
 constexpr int kWarpMma = 17;
-constexpr int kWarpConv = 18;  // two warps, INT8 KV cache only
+constexpr int kWarpConv = 18;  // two converter warps (modes 1 and 2)
+// Operand modes: Q8/K8 and scales given (quantised once before the call),
+// the INT8 KV cache (K8/V8 given, fp16 copies made on chip), or Q8/K8 and
+// their scales made on chip from Q/K for INT8-routed tiles only.
+constexpr int kModeGiven = 0, kModeKV8 = 1, kModeOnChip = 2;
 // 16 softmax warps, producer, MMA issuer (+ two converter warps)
-__host__ __device__ constexpr int threads_of(bool kv8) { return kv8 ? 640 : 576; }
+__host__ __device__ constexpr int threads_of(int mode) {
+  return mode != kModeGiven ? 640 : 576;
+}
 constexpr int kSmemBudget = 232448;  // max dynamic smem per block on sm_100
 constexpr uint32_t kKindF16 = 1, kKindI8 = 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the
@@ -57,8 +64,9 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the
 
 __host__ __device__ constexpr int align1k(int x) { return (x + 1023) & ~1023; }
 
-template <int D, bool DUAL, bool KV8>
+template <int D, bool DUAL, int MODE>
 struct Cfg {
+  static constexpr bool KV8 = MODE == kModeKV8;
   // DUAL (64-row routing words): a 128-row query tile may need both paths
   // for the same keys, so S has an fp16 and an int8 region and the CTA
   // holds one query tile.
@@ -83,7 +91,7 @@ struct Cfg {
   static constexpr int kRedBytes = 4096;  // max / sum exchange [tile][2][2][128]
   static constexpr int kBarBytes = 512;
   static constexpr int kAvail =
-      kSmemBudget - 1024 - kBarBytes - kRedBytes - kRing0;
+      kSmemBudget - 1024 - kBarBytes - kRedBytes - 128 - kRing0;
   // Two V slots (P V of every query tile must finish before a V slot
   // frees), then as many K slots as fit (at most 3).
   static constexpr int kVStages = 2;
@@ -92,7 +100,12 @@ struct Cfg {
   static_assert(kKStages >= 1, "shared memory too small");
   static constexpr int kVRing0 = kRing0 + kKStages * kKSlotBytes;
   static constexpr int kRedOff = kVRing0 + kVStages * kVSlotBytes;
-  static constexpr int kBarOff = kRedOff + kRedBytes;
+  // on-chip quantisation: Q scales [2], K-scale ring [8], converter max
+  // exchange [2][2]
+  static constexpr int kAuxOff = kRedOff + kRedBytes;
+  static constexpr int kAuxBytes = 128;
+  static constexpr int kSkRing = 8;
+  static constexpr int kBarOff = kAuxOff + kAuxBytes;
   static constexpr int kSmem = kBarOff + kBarBytes + 1024;  // + align slack
   static_assert(kSmem - 1024 <= kSmemBudget, "shared memory overflow");
   // TMEM columns of query tile t start at t * kTileCols: the S region(s),
@@ -124,7 +137,12 @@ struct Cfg {
   static constexpr int kBarOStage = kBarRed + 4;       // [tile]
   static constexpr int kBarKConv = kBarOStage + 2;     // [K slot]
   static constexpr int kBarVConv = kBarKConv + kKStages;  // [V slot]
-  static constexpr int kBarDrain = kBarVConv + kVStages;
+  // on-chip quantisation: Q8 of a tile made, K scale of a key tile made,
+  // converter-warp max exchange
+  static constexpr int kBarQConv = kBarVConv + kVStages;  // [tile]
+  static constexpr int kBarSK = kBarQConv + 2;            // [ring slot]
+  static constexpr int kBarCvX = kBarSK + kSkRing;
+  static constexpr int kBarDrain = kBarCvX + 1;
   static constexpr int kNumBars = kBarDrain + 1;
   static_assert(kNumBars * 8 + 16 <= kBarBytes, "barrier area");
 };
@@ -292,6 +310,49 @@ __device__ __forceinline__ void convert_row(const uint8_t* src, uint32_t sm,
   }
 }
 
+// Largest |x| of row rr of an fp16 tile stored as D/64 chunks of
+// [128 rows][128 B] with the 128-byte swizzle.
+template <int D>
+__device__ __forceinline__ float row_absmax_f16(const uint8_t* tile, int rr) {
+  __half2 m = __float2half2_rn(0.0f);
+#pragma unroll
+  for (int u = 0; u < D / 8; ++u) {
+    const uint32_t o = (u / 8) * 128 * 128 + rr * 128 + (u % 8) * 16;
+    const uint4 v = *reinterpret_cast<const uint4*>(tile + swz(o, 7));
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) m = __hmax2(m, __habs2(h[e]));
+  }
+  return fmaxf(__low2float(m), __high2float(m));
+}
+
+// Codes of row rr of that fp16 tile into an INT8 tile of D-byte rows with
+// the swizzle of mask sm (the layout the INT8 MMA reads), scale s, 1/s = r;
+// zero: the block is all zeros (codes 0).
+template <int D>
+__device__ __forceinline__ void quant_row(const uint8_t* tile16,
+                                          uint8_t* tile8, uint32_t sm, int rr,
+                                          float s, float r, bool zero) {
+#pragma unroll
+  for (int v = 0; v < D / 16; ++v) {
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int hu = 0; hu < 2; ++hu) {
+      const int u = 2 * v + hu;
+      const uint32_t o = (u / 8) * 128 * 128 + rr * 128 + (u % 8) * 16;
+      const uint4 x = *reinterpret_cast<const uint4*>(tile16 + swz(o, 7));
+      const __half* h = reinterpret_cast<const __half*>(&x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int q = zero ? 0 : quant_code(__half2float(h[e]), s, r);
+        w[2 * hu + e / 4] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (e % 4));
+      }
+    }
+    *reinterpret_cast<uint4*>(tile8 + swz(rr * D + v * 16, sm)) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 // Routing state of one 128-row query tile.
 struct TileRoute {
   uint64_t w0, w1;  // words of rows 0..63 / 64..127 (equal unless DUAL)
@@ -299,10 +360,12 @@ struct TileRoute {
   int n_last;       // last legal 128-key tile (-1: no rows)
 };
 
-template <int D, bool DUAL, bool KV8>
-__global__ void __launch_bounds__(threads_of(KV8), 1)
+template <int D, bool DUAL, int MODE>
+__global__ void __launch_bounds__(threads_of(MODE), 1)
     attn_fwd_kernel(const __grid_constant__ AttnParams p) {
-  using C = Cfg<D, DUAL, KV8>;
+  using C = Cfg<D, DUAL, MODE>;
+  constexpr bool KV8 = MODE == kModeKV8;
+  constexpr bool QF = MODE == kModeOnChip;
   constexpr int kQT = C::kQT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -403,11 +466,14 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
       mbar_init(&bars[C::kBarRed + 2 * i], 8);
       mbar_init(&bars[C::kBarRed + 2 * i + 1], 8);
     }
-    if (KV8) {
+    if (KV8 || QF) {
       for (int s = 0; s < C::kKStages; ++s)
         mbar_init(&bars[C::kBarKConv + s], 2);  // the two converter warps
       for (int s = 0; s < C::kVStages; ++s)
         mbar_init(&bars[C::kBarVConv + s], 2);
+      for (int i = 0; i < 2; ++i) mbar_init(&bars[C::kBarQConv + i], 2);
+      for (int i = 0; i < C::kSkRing; ++i) mbar_init(&bars[C::kBarSK + i], 2);
+      mbar_init(&bars[C::kBarCvX], 2);
     }
     mbar_init(&bars[C::kBarDrain], 1);
     *abort_flag = 0;
@@ -421,7 +487,7 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
     }
-    if (routed) {  // the INT8 maps are left empty in FP16-only mode
+    if (routed && !QF) {  // the INT8 maps are empty in FP16-only mode
       tma_prefetch_desc(&p.tm_q8);
       if (!KV8) tma_prefetch_desc(&p.tm_k8);
     }
@@ -458,7 +524,10 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
         return k;
       };
       uint32_t qbytes = 0;
-      const uint32_t need[2] = {need_of(rt0), need_of(rt1)};
+      uint32_t need[2] = {need_of(rt0), need_of(rt1)};
+      // On-chip quantisation makes Q8 from Q: fetch Q for every tile.
+      if (QF)
+        for (int t = 0; t < 2; ++t) need[t] = need[t] ? kKindF16 : 0u;
       for (int t = 0; t < kQT; ++t)
         qbytes += ((need[t] & kKindF16) ? C::kQBytes : 0) +
                   ((need[t] & kKindI8) ? C::kQ8Bytes : 0);
@@ -487,8 +556,10 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
         uint32_t kinds = 0;
         for (int t = 0; t < kQT; ++t)
           kinds |= kinds_of(t, n, 0) | kinds_of(t, n, 1);
-        // The INT8 cache only holds K8 (the converters make the fp16 copy).
+        // The INT8 cache only holds K8 (the converters make the fp16 copy);
+        // on-chip quantisation makes K8 from K.
         if (KV8) kinds = kKindI8;
+        if (QF) kinds = kKindF16;
         mbar_arrive_expect_tx(&bars[C::kBarK + ks],
                               ((kinds & kKindF16) ? C::kK16Bytes : 0) +
                                   ((kinds & kKindI8) ? C::kK8Bytes : 0));
@@ -543,6 +614,7 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
       bool ok = mbar_wait(&bars[C::kBarQ], 0, abort_flag);
       tc_fence_after();
 
+      bool q8_ready0 = false, q8_ready1 = false;  // on-chip Q8 seen
       // S_t(n) = Q_t K(n)^T, each 64-key half on the path(s) it routes to.
       auto issue_qk = [&](int t, int n) -> bool {
         if (n > rt(t).n_last) return true;
@@ -559,10 +631,22 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
                                   ((k1 & kKindF16) ? 2u : 0u);
         const uint32_t halves8 = ((k0 & kKindI8) ? 1u : 0u) |
                                  ((k1 & kKindI8) ? 2u : 0u);
-        if (halves16 && KV8 &&
+        // With converter warps, every key tile waits for them (the fp16 copy
+        // of an INT8-cache K tile, or the on-chip K8): the K slot may only
+        // free after they passed it, so they never miss a phase of its
+        // full barrier.
+        if ((KV8 || QF) &&
             !mbar_wait(&bars[C::kBarKConv + s], (n / C::kKStages) & 1,
                        abort_flag))
           return false;
+        // On-chip quantisation: the converters' Q8 of this tile (once).
+        if (QF && halves8) {
+          bool& qdone = t ? q8_ready1 : q8_ready0;
+          if (!qdone && !mbar_wait(&bars[C::kBarQConv + t], 0, abort_flag))
+            return false;
+          qdone = true;
+        }
+        if (KV8 || QF) tc_fence_after();
         if (halves16) {
           const uint32_t q16 = smem_u32(sQ(t));
           const bool both = halves16 == 3u;
@@ -692,6 +776,104 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
       }
       if (!ok) fail();
     }
+    if (QF) {
+      // =================== on-chip quantisation (2 warps) ===================
+      // Q8 of each query tile once, then K8 of each key tile that some row
+      // routes to INT8, with the quantiser's definition over the block's
+      // rows inside the sequence (a 128-row tile is one 128-token block).
+      // Each thread quantises whole rows (ct and ct + 64); the block max
+      // combines the two warps through shared memory.
+      const int cw = warp - kWarpConv;
+      const int ct = cw * 32 + lane;
+      float* aux = reinterpret_cast<float*>(smem + C::kAuxOff);
+      float* sq_s = aux;          // [2] Q scale of each query tile
+      float* sk_ring = aux + 2;   // [kSkRing] K scale of key tile n % ring
+      float* xmax = aux + 2 + C::kSkRing;  // [2 slots][2 warps]
+      constexpr uint32_t i8_swz = D == 128 ? 7u : 3u;
+      uint32_t xu = 0;  // max exchanges so far
+      bool ok = true;
+      auto block_max = [&](float v, bool& good) -> float {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+        float* slot = xmax + (xu & 1) * 2;
+        if (lane == 0) slot[cw] = v;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[C::kBarCvX]);
+        const bool got = mbar_wait(&bars[C::kBarCvX], xu & 1, abort_flag);
+        good = __all_sync(0xffffffffu, got);
+        const float other = slot[1 - cw];
+        ++xu;
+        return fmaxf(v, other);
+      };
+      const bool got_q = mbar_wait(&bars[C::kBarQ], 0, abort_flag);
+      ok = __all_sync(0xffffffffu, got_q);
+      for (int t = 0; t < kQT && ok; ++t) {
+        const TileRoute R = rt(t);
+        bool any8 = false;
+        for (int n = 0; n <= R.n_last; ++n)
+          any8 |= ((kinds_of(t, n, 0) | kinds_of(t, n, 1)) & kKindI8) != 0;
+        float sq = 0.0f;
+        if (any8) {
+          const int row0 = row_base + t * kBM;
+          float local = 0.0f;
+          for (int rr = ct; rr < kBM; rr += 64)
+            if (row0 + rr < len) local = fmaxf(local, row_absmax_f16<D>(sQ(t), rr));
+          bool good = true;
+          const float amax = block_max(local, good);
+          if (!good) {
+            ok = false;
+            break;
+          }
+          sq = __fdiv_rn(amax, 127.0f);
+          const float rcp = amax != 0.0f ? __frcp_rn(sq) : 0.0f;
+          for (int rr = ct; rr < kBM; rr += 64)
+            quant_row<D>(sQ(t), sQ8(t), i8_swz, rr, sq, rcp, amax == 0.0f);
+          fence_proxy_async_smem();
+        }
+        if (ct == 0) sq_s[t] = sq;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[C::kBarQConv + t]);
+      }
+      for (int n = 0; n <= n_end && ok; ++n) {
+        const int ks = n % C::kKStages;
+        const bool got_k = mbar_wait(&bars[C::kBarK + ks],
+                                     (n / C::kKStages) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got_k)) {
+          ok = false;
+          break;
+        }
+        uint32_t kinds = 0;
+        for (int t = 0; t < kQT; ++t)
+          kinds |= kinds_of(t, n, 0) | kinds_of(t, n, 1);
+        float sk = 0.0f;
+        if (kinds & kKindI8) {
+          uint8_t* kp = kslot(ks);
+          float local = 0.0f;
+          for (int rr = ct; rr < kBN; rr += 64)
+            if (n * kBN + rr < len) local = fmaxf(local, row_absmax_f16<D>(kp, rr));
+          bool good = true;
+          const float amax = block_max(local, good);
+          if (!good) {
+            ok = false;
+            break;
+          }
+          sk = __fdiv_rn(amax, 127.0f);
+          const float rcp = amax != 0.0f ? __frcp_rn(sk) : 0.0f;
+          for (int rr = ct; rr < kBN; rr += 64)
+            quant_row<D>(kp, kp + C::kK8Off, i8_swz, rr, sk, rcp,
+                         amax == 0.0f);
+          fence_proxy_async_smem();
+        }
+        if (ct == 0) sk_ring[n % C::kSkRing] = sk;
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bars[C::kBarKConv + ks]);
+          mbar_arrive(&bars[C::kBarSK + n % C::kSkRing]);
+        }
+      }
+      if (!ok) fail();
+    }
   } else {
     // =================== softmax warps 0-15 ===================
     // Warpgroups 2t and 2t+1 serve query tile t: thread = score row = TMEM
@@ -726,7 +908,10 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
         const int blk = (n * kBN + c0) / p.quant_block_k;
         return kscale[min(blk, p.nbk - 1)];
       };
-      float sk_next = ((routed || KV8) && R.n_last >= 0) ? ksc(0) : 0.0f;
+      float sk_next =
+          ((routed || KV8) && !QF && R.n_last >= 0) ? ksc(0) : 0.0f;
+      // On-chip quantisation: the converters' scales in shared memory.
+      const float* aux = reinterpret_cast<const float*>(smem + C::kAuxOff);
       // INT8 KV cache: the V scale's mantissa factor f in [1, 2) of this
       // thread's 64 keys (the converters put its power of two into V).
       const float* vscale =
@@ -742,11 +927,17 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
       float fv_next = (KV8 && R.n_last >= 0) ? vfrac(0) : 1.0f;
       // softmax scale (log2 units) times the Q block scale of this row: the
       // INT8 path's S c = (Q8 K8^T) sq sk scale log2(e)
-      const float cq =
-          routed ? p.scale_log2 *
-                       p.q_scale[(static_cast<size_t>(h) * p.batch + b) * p.nbq +
-                                 key_lim / p.quant_block_q]
-                 : 0.0f;
+      float cq =
+          (routed && !QF)
+              ? p.scale_log2 *
+                    p.q_scale[(static_cast<size_t>(h) * p.batch + b) * p.nbq +
+                              key_lim / p.quant_block_q]
+              : 0.0f;
+      if (QF && routed && R.n_last >= 0) {
+        const bool got = mbar_wait(&bars[C::kBarQConv + t], 0, abort_flag);
+        ok = __all_sync(0xffffffffu, got);
+        cq = p.scale_log2 * aux[t];
+      }
       // running max and (this warpgroup's) sum of the row
       float m_run = -CUDART_INF_F, l_run = 0.0f;
       uint32_t u = 0;  // exchanges so far: slot and parity
@@ -765,9 +956,19 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
         return other;
       };
 
-      for (int n = 0; n <= R.n_last; ++n) {
-        const float sk = sk_next;
-        if ((routed || KV8) && n < R.n_last) sk_next = ksc(n + 1);
+      for (int n = 0; n <= R.n_last && ok; ++n) {
+        float sk = sk_next;
+        if ((routed || KV8) && !QF && n < R.n_last) sk_next = ksc(n + 1);
+        if (QF && routed) {
+          const int slot = n % C::kSkRing;
+          const bool got = mbar_wait(&bars[C::kBarSK + slot],
+                                     (n / C::kSkRing) & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, got)) {
+            ok = false;
+            break;
+          }
+          sk = aux[2 + slot];
+        }
         const float fv = fv_next;
         if (KV8 && n < R.n_last) fv_next = vfrac(n + 1);
         // Exits stay warp-uniform: the tcgen05.ld/st below are .sync.aligned.
@@ -964,34 +1165,44 @@ __global__ void __launch_bounds__(threads_of(KV8), 1)
   if (warp == kWarpMma) tmem_dealloc(tmem, C::kTmemCols);
 }
 
-template <int D, bool DUAL, bool KV8>
+template <int D, bool DUAL, int MODE>
 cudaError_t launch_one(const AttnParams& p, cudaStream_t stream) {
-  using C = Cfg<D, DUAL, KV8>;
-  auto kern = attn_fwd_kernel<D, DUAL, KV8>;
+  using C = Cfg<D, DUAL, MODE>;
+  auto kern = attn_fwd_kernel<D, DUAL, MODE>;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const int groups = (p.max_seqlen + C::kQT * kBM - 1) / (C::kQT * kBM);
   dim3 grid(p.hq, groups, p.batch);
-  kern<<<grid, threads_of(KV8), C::kSmem, stream>>>(p);
+  kern<<<grid, threads_of(MODE), C::kSmem, stream>>>(p);
   return cudaGetLastError();
+}
+
+template <int D, int MODE>
+cudaError_t launch_dm(const AttnParams& p, const AttnLaunchShape& s,
+                      cudaStream_t stream) {
+  return s.dual ? launch_one<D, true, MODE>(p, stream)
+                : launch_one<D, false, MODE>(p, stream);
 }
 
 template <int D>
 cudaError_t launch_d(const AttnParams& p, const AttnLaunchShape& s,
                      cudaStream_t stream) {
-  if (s.kv8)
-    return s.dual ? launch_one<D, true, true>(p, stream)
-                  : launch_one<D, false, true>(p, stream);
-  return s.dual ? launch_one<D, true, false>(p, stream)
-                : launch_one<D, false, false>(p, stream);
+  if (s.mode == kModeKV8) return launch_dm<D, kModeKV8>(p, s, stream);
+  if (s.mode == kModeOnChip) return launch_dm<D, kModeOnChip>(p, s, stream);
+  return launch_dm<D, kModeGiven>(p, s, stream);
+}
+
+template <int D, int MODE>
+int smem_dm(const AttnLaunchShape& s) {
+  return s.dual ? Cfg<D, true, MODE>::kSmem : Cfg<D, false, MODE>::kSmem;
 }
 
 template <int D>
 int smem_d(const AttnLaunchShape& s) {
-  if (s.kv8)
-    return s.dual ? Cfg<D, true, true>::kSmem : Cfg<D, false, true>::kSmem;
-  return s.dual ? Cfg<D, true, false>::kSmem : Cfg<D, false, false>::kSmem;
+  if (s.mode == kModeKV8) return smem_dm<D, kModeKV8>(s);
+  if (s.mode == kModeOnChip) return smem_dm<D, kModeOnChip>(s);
+  return smem_dm<D, kModeGiven>(s);
 }
 
 }  // namespace

@@ -76,7 +76,9 @@ struct AttnParams {
 struct AttnLaunchShape {
   int head_dim;
   bool dual;  // routing rows of 64 inside 128-row compute tiles
-  bool kv8;   // K and V arrive as an INT8 cache (k8, v8 + block scales)
+  // 0: Q8/K8 + scales given; 1: INT8 KV cache (k8, v8 + block scales);
+  // 2: Q8/K8 + scales made on chip for INT8-routed tiles
+  int mode;
 };
 
 cudaError_t launch_attn_prefill(const AttnParams& p, const AttnLaunchShape& s,

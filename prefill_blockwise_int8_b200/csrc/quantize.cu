@@ -16,28 +16,12 @@
 #include <stdint.h>
 
 #include "internal.h"
+#include "quant_code.cuh"
 
 namespace tilemix {
 namespace {
 
 constexpr int kQThreads = 256;
-
-// code = rint(fl(x / s)) without a division per element: y = x * fl(1/s)
-// lies within a few ulp of fl(x / s) (|y| <= 128, so within 2^-15), hence
-// both round to the same integer unless y is within that distance of a
-// half-integer; those rare elements take the IEEE division.
-__device__ __forceinline__ int quant_code(float x, float s, float r) {
-  const float y = x * r;
-  const float t = rintf(y);
-  const float frac = fabsf(y - t);  // in [0, 0.5] (+ rounding)
-  int q;
-  if (frac < 0.5f - 0x1p-13f) {
-    q = static_cast<int>(t);
-  } else {
-    q = __float2int_rn(__fdiv_rn(x, s));
-  }
-  return max(-127, min(127, q));
-}
 
 // VPT 16-byte vectors (8 halves) per thread; VPR vectors per row (d / 8),
 // 0 = taken from vpr_rt at run time.

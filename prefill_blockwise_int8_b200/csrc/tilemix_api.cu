@@ -224,7 +224,9 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   if (a->causal != 1)
     return fail(TILEMIX_ERR_UNSUPPORTED, "attn: only causal attention is built");
   const bool fp16_only = (a->flags & TILEMIX_FLAG_FP16_ONLY) != 0;
-  if (a->flags & ~TILEMIX_FLAG_FP16_ONLY)
+  // With every tile FP16 there is nothing to quantise on chip.
+  const bool on_chip = !fp16_only && (a->flags & TILEMIX_FLAG_QUANT_ON_CHIP) != 0;
+  if (a->flags & ~(TILEMIX_FLAG_FP16_ONLY | TILEMIX_FLAG_QUANT_ON_CHIP))
     return fail(TILEMIX_ERR_INVALID_ARG, "attn: unknown flag bits 0x%x",
                 a->flags);
   if (a->kv_format != TILEMIX_KV_FP16 && a->kv_format != TILEMIX_KV_INT8)
@@ -271,10 +273,19 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   if (kv8 && (!a->k8 || !a->k_scale || !a->v8 || !a->v_scale))
     return fail(TILEMIX_ERR_INVALID_ARG,
                 "attn: the INT8 KV cache needs k8, k_scale, v8 and v_scale");
-  if (!fp16_only && (!a->mask || !a->q8 || !a->q_scale || !a->k8 || !a->k_scale))
+  if (on_chip && kv8)
+    return fail(TILEMIX_ERR_UNSUPPORTED,
+                "attn: on-chip quantisation needs the FP16 KV format");
+  if (on_chip && (qbq != 128 || qbk != 128))
+    return fail(TILEMIX_ERR_UNSUPPORTED,
+                "attn: on-chip quantisation needs 128-token quantisation blocks");
+  if (on_chip && !a->mask)
+    return fail(TILEMIX_ERR_INVALID_ARG, "attn: mask is required");
+  if (!fp16_only && !on_chip &&
+      (!a->mask || !a->q8 || !a->q_scale || !a->k8 || !a->k_scale))
     return fail(TILEMIX_ERR_INVALID_ARG,
                 "attn: mask, q8, q_scale, k8 and k_scale are required unless "
-                "TILEMIX_FLAG_FP16_ONLY is set");
+                "TILEMIX_FLAG_FP16_ONLY or TILEMIX_FLAG_QUANT_ON_CHIP is set");
   if (!aligned(a->q, 16) || (a->k && !aligned(a->k, 16)) ||
       (a->v && !aligned(a->v, 16)) || (a->v8 && !aligned(a->v8, 16)) ||
       (a->v_scale && !aligned(a->v_scale, 4)) ||
@@ -311,12 +322,12 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
                     a->hkv, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
            make_map(&p.tm_v, a->v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
                     a->hkv, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (maps && !fp16_only)
+  if (maps && !fp16_only && !on_chip)
     maps = make_map(&p.tm_q8, a->q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
                     a->hq, d, 128, i8sw);
   // The INT8 cache always feeds K8 (the INT8 path, or converted to fp16 on
   // chip for FP16 groups) and V8 (converted to fp16 on chip).
-  if (maps && (kv8 || !fp16_only))
+  if (maps && (kv8 || (!fp16_only && !on_chip)))
     maps = make_map(&p.tm_k8, a->k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
                     a->hkv, d, 128, i8sw);
   if (maps && kv8)
@@ -327,8 +338,8 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   p.cu_seqlens = a->cu_seqlens;
   p.head_map = a->head_map;
   p.mask = fp16_only ? nullptr : a->mask;
-  p.q_scale = fp16_only ? nullptr : a->q_scale;
-  p.k_scale = (fp16_only && !kv8) ? nullptr : a->k_scale;
+  p.q_scale = (fp16_only || on_chip) ? nullptr : a->q_scale;
+  p.k_scale = ((fp16_only && !kv8) || on_chip) ? nullptr : a->k_scale;
   p.v_scale = kv8 ? a->v_scale : nullptr;
   p.out = static_cast<uint16_t*>(a->out);
   p.lse = a->lse;
@@ -355,7 +366,7 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
       a->softmax_scale > 0.0f ? a->softmax_scale : 1.0f / std::sqrt(float(d));
   p.scale_log2 = scale * 1.4426950408889634f;
 
-  tilemix::AttnLaunchShape shape{d, a->block_m == 64, kv8};
+  tilemix::AttnLaunchShape shape{d, a->block_m == 64, kv8 ? 1 : (on_chip ? 2 : 0)};
   cudaError_t e = tilemix::launch_attn_prefill(p, shape, stream);
   if (e != cudaSuccess)
     return fail(TILEMIX_ERR_CUDA, "attn launch: %s", cudaGetErrorString(e));

@@ -28,7 +28,7 @@ def dev_tensor(a):
 
 
 def run_gpu(inp, *, fp16_only=False, want_lse=False, want_dump=False,
-            head_map=None, stream=None, route=None):
+            head_map=None, stream=None, route=None, on_chip=False):
     """Quantise Q and K, pack the routing words and run attention on the GPU.
     Returns numpy copies of everything the path produced."""
     torch = torch_mod()
@@ -64,7 +64,9 @@ def run_gpu(inp, *, fp16_only=False, want_lse=False, want_dump=False,
     hm = dev_tensor(np.asarray(head_map, np.int32)) if head_map is not None \
         else None
     out = tm.tilemix_attn_prefill(
-        q, k, v, cu, ms, q8=q8, q_scale=sq, k8=k8, k_scale=sk, v8=v8,
+        q, k, v, cu, ms, q8=None if on_chip else q8,
+        q_scale=None if on_chip else sq, k8=None if on_chip else k8,
+        k_scale=None if on_chip else sk, v8=v8, quant_on_chip=on_chip,
         v_scale=sv, mask=mask, block_m=w.block_m, block_n=w.block_n, group=g,
         quant_block_q=w.quant_block_q, quant_block_k=w.quant_block_k,
         head_map=hm, fp16_only=fp16_only, lse=lse, qk_dump=dump,

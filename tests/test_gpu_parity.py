@@ -342,3 +342,52 @@ def test_route_template_through_attention(tm):
     assert got["status"] == 0
     ref, _ = run_oracle(inp, route=route)
     compare(got["out"], ref)
+
+
+# ----------------------------------------------------------------------------
+# on-chip quantisation: identical to quantise-once, element for element
+# ----------------------------------------------------------------------------
+
+ON_CHIP_CASES = {
+    "d128_bn64_two_seqs": ([700, 300, 1], dict()),
+    "d128_bn128_g2": ([1500], dict(bn=128, g=2, recipe="exact", cov=0.5)),
+    "d64_bm64_dual": ([400], dict(d=64, bm=64, bn=64, recipe="bernoulli", cov=0.5)),
+    "gqa7_all_int8": ([520], dict(hq=7, hkv=1, recipe="exact", cov=1.0)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(ON_CHIP_CASES))
+def test_quant_on_chip_equals_quantise_once(tm, name):
+    lens, kw = ON_CHIP_CASES[name]
+    inp = small(lens, **kw)
+    once = run_gpu(inp, want_lse=True, want_dump=True)
+    chip = run_gpu(inp, want_lse=True, want_dump=True, on_chip=True)
+    assert once["status"] == 0 and chip["status"] == 0
+    assert np.array_equal(chip["dump"], once["dump"])
+    assert np.array_equal(chip["out"], once["out"])
+    assert np.array_equal(chip["lse"], once["lse"])
+    ref, _ = run_oracle(inp)
+    compare(chip["out"], ref)
+
+
+def test_quant_on_chip_full_size_sampled_rows(tm):
+    w = W.LLAMA32_3B_4K
+    inp = W.make(w)
+    got = run_gpu(inp, on_chip=True)
+    assert got["status"] == 0
+    rows = sample_rows(inp["seqlens"], inp["cu_seqlens"], per_seq=16,
+                       block=w.block_m)
+    ref, _ = run_oracle(inp, rows=rows)
+    compare(got["out"], ref, rows=rows)
+
+
+def test_quant_on_chip_host_checks(tm):
+    inp = small([256])
+    q = dev_tensor(inp["q"])
+    with pytest.raises(tm.TilemixError):  # 64-token K blocks are not tiles
+        tm.tilemix_attn_prefill(q, dev_tensor(inp["k"]), dev_tensor(inp["v"]),
+                                dev_tensor(inp["cu_seqlens"]), 256,
+                                mask=torch.zeros((1, 2, 2), dtype=torch.int64,
+                                                 device="cuda"),
+                                block_m=128, block_n=64, quant_block_k=64,
+                                quant_on_chip=True)
