@@ -5,9 +5,11 @@ the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import
 this package.  The product path (``prefill_blockwise_int8_b200``) never
 imports it and shares no code with it.
 
-The arithmetic lives in ``tilemix_oracle.c`` (plain C, fp64, exact integer
-dots); this module compiles it with gcc and marshals numpy arrays.  Each C
-function cites the passage of the TileMix pages it restates.
+The attention, quantiser and packer arithmetic lives in
+``tilemix_oracle.c`` (plain C, fp64, exact integer dots); this module
+compiles it with gcc and marshals numpy arrays.  Each C function cites the
+passage of the TileMix pages it restates.  The routing templates and the
+adaptive routing statistic are plain Python below, in exact integers.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (closed forms, dense textbook attention in fp64, library attention, brute
@@ -307,6 +309,82 @@ def route_template(layout, int8_permille: int, seed: int, cu_seqlens,
                     keys.append((_priority(code, j, G - 1 - j) << 32) | h)
                 # FP16: the k_fp16 largest keys, ties to the smaller index
                 order = sorted(range(G), key=lambda i: (-keys[i], i))
+                for j in order[k_fp16:]:
+                    out[b, hk, m, j] = 1
+    return out
+
+
+def fp16_fixed(x) -> np.ndarray:
+    """Exact integer value of fp16 numbers times 2^24 (int64): every finite
+    fp16 value is an integer multiple of 2^-24 below 2^16 in magnitude."""
+    return (np.asarray(x, dtype=np.float16).astype(np.float64)
+            * 2.0 ** 24).astype(np.int64)
+
+
+def route_adaptive_statistic(q, k, cu_seqlens, max_seqlen: int, block_m: int,
+                             block_n: int, group: int, head_map=None):
+    """Adaptive-routing statistic I[b][hk][m] = list over the row's G legal
+    groups j of (sum of the row's queries over hk's heads) . (sum of group j's
+    keys), in exact integers (fp16 values scaled by 2^24).
+
+    Reading of the TileMix pages' remark that the kernel interface takes
+    adaptive routing policies (paperlayer summary, Limitations) and of the
+    heavy-hitter analysis (appendix G.5): the statistic equals 2^48 times the
+    sum of all raw logits between the row's queries and the group's keys."""
+    q = np.asarray(q, dtype=np.float16)
+    k = np.asarray(k, dtype=np.float16)
+    _, hq, _ = q.shape
+    hkv = k.shape[1]
+    hmap = [h // (hq // hkv) for h in range(hq)] if head_map is None \
+        else [int(x) for x in head_map]
+    cu = [int(x) for x in cu_seqlens]
+    tm = -(-max_seqlen // block_m)
+    xq, xk = fp16_fixed(q), fp16_fixed(k)
+    kpg = group * block_n
+    stats = []
+    for b in range(len(cu) - 1):
+        start, L = cu[b], cu[b + 1] - cu[b]
+        per_b = []
+        for hk in range(hkv):
+            heads = [h for h in range(hq) if hmap[h] == hk]
+            per_h = []
+            for m in range(tm):
+                if m * block_m >= L:
+                    per_h.append([])
+                    continue
+                r0, r1 = start + m * block_m, start + min((m + 1) * block_m, L)
+                G = ((min((m + 1) * block_m, L) - 1) // block_n) // group + 1
+                sq = xq[r0:r1][:, heads, :].sum(axis=(0, 1)).astype(object) \
+                    if heads else np.zeros(q.shape[2], dtype=object)
+                row = []
+                for j in range(G):
+                    k0, k1 = start + j * kpg, start + min((j + 1) * kpg, L)
+                    sk = xk[k0:k1, hk, :].sum(axis=0).astype(object)
+                    row.append(int(np.dot(sq, sk)))
+                per_h.append(row)
+            per_b.append(per_h)
+        stats.append(per_b)
+    return stats
+
+
+def route_adaptive(q, k, cu_seqlens, max_seqlen: int, block_m: int,
+                   block_n: int, group: int, int8_permille: int,
+                   head_map=None) -> np.ndarray:
+    """uint8 [batch, hkv, ceil(max_seqlen / block_m), 64], 1 = INT8: per
+    legal row, the G - k_int8 groups with the largest statistic stay FP16
+    (ties to the smaller group index), k_int8 = round-half-up of
+    permille * G / 1000 as for the routing templates."""
+    stats = route_adaptive_statistic(q, k, cu_seqlens, max_seqlen, block_m,
+                                     block_n, group, head_map)
+    hkv = np.asarray(k).shape[1]
+    tm = -(-max_seqlen // block_m)
+    out = np.zeros((len(stats), hkv, tm, 64), dtype=np.uint8)
+    for b, per_b in enumerate(stats):
+        for hk, per_h in enumerate(per_b):
+            for m, imp in enumerate(per_h):
+                G = len(imp)
+                k_fp16 = G - (int8_permille * G + 500) // 1000
+                order = sorted(range(G), key=lambda j: (-imp[j], j))
                 for j in order[k_fp16:]:
                     out[b, hk, m, j] = 1
     return out

@@ -467,3 +467,113 @@ def test_splitmix64_is_a_bijection_on_a_sample():
     vals = {oracle.splitmix64(x) for x in range(1 << 14)}
     assert len(vals) == 1 << 14
     assert all(0 <= v < (1 << 64) for v in vals)
+
+
+# ----------------------------------------------------------------------------
+# adaptive routing: the statistic is the exact sum of raw logits (x 2^48)
+# between a query-tile row and a key group; FP16 goes to the largest
+# ----------------------------------------------------------------------------
+
+def _adaptive_case(seed=3, lens=(13, 21, 0, 6), hq=4, hkv=2, d=8):
+    rng = np.random.default_rng(seed)
+    T = int(sum(lens))
+    q = (rng.standard_normal((T, hq, d)) * 3).astype(np.float16)
+    k = (rng.standard_normal((T, hkv, d)) * 3).astype(np.float16)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return q, k, cu, int(max(lens))
+
+
+def test_adaptive_statistic_is_the_brute_force_logit_sum():
+    from fractions import Fraction
+    q, k, cu, ms = _adaptive_case()
+    bm, bn, g, hq, hkv = 4, 3, 2, 4, 2
+    stats = oracle.route_adaptive_statistic(q, k, cu, ms, bm, bn, g)
+    for b in range(len(cu) - 1):
+        s0, L = int(cu[b]), int(cu[b + 1] - cu[b])
+        for hk in range(hkv):
+            for m, row in enumerate(stats[b][hk]):
+                rows = range(m * bm, min((m + 1) * bm, L))
+                assert len(row) == (((rows[-1] // bn) // g) + 1 if rows else 0)
+                for j, got in enumerate(row):
+                    keys = range(j * g * bn, min((j + 1) * g * bn, L))
+                    want = Fraction(0)
+                    for i in rows:
+                        for h in range(hq):
+                            if h // (hq // hkv) != hk:
+                                continue
+                            for key in keys:
+                                for c in range(q.shape[2]):
+                                    want += Fraction(float(q[s0 + i, h, c])) * \
+                                        Fraction(float(k[s0 + key, hk, c]))
+                    assert want * 2 ** 48 == got
+
+
+def test_adaptive_keeps_the_heaviest_groups_fp16():
+    # positive queries; keys of group j carry j + 1 in channel 0, so the
+    # logit sums grow with j and FP16 must go to the last groups of each row
+    bm = bn = 16
+    L, hq, hkv, d = 8 * 16, 2, 1, 8
+    q = np.zeros((L, hq, d), np.float16)
+    q[:, :, 0] = 1.0
+    k = np.zeros((L, hkv, d), np.float16)
+    k[:, 0, 0] = (np.arange(L) // bn + 1).astype(np.float16)
+    cu = np.array([0, L], np.int32)
+    for permille in (0, 250, 500, 750, 1000):
+        r = oracle.route_adaptive(q, k, cu, L, bm, bn, 1, permille)
+        for m in range(L // bm):
+            G = m + 1
+            k8 = (permille * G + 500) // 1000
+            want = np.zeros(64, np.uint8)
+            want[:k8] = 1          # the lightest groups are the first ones
+            assert np.array_equal(r[0, 0, m], want), (permille, m)
+
+
+def test_adaptive_ties_go_to_the_smaller_group():
+    q, k, cu, ms = _adaptive_case()
+    q[:] = 0                   # every statistic 0: pure tie
+    r = oracle.route_adaptive(q, k, cu, ms, 4, 3, 1, 500)
+    for b in range(len(cu) - 1):
+        L = int(cu[b + 1] - cu[b])
+        for m in range(-(-L // 4)):
+            G = (min((m + 1) * 4, L) - 1) // 3 + 1
+            k8 = (500 * G + 500) // 1000
+            want = np.zeros(64, np.uint8)
+            want[G - k8:G] = 1
+            assert np.array_equal(r[b, 0, m], want)
+
+
+@pytest.mark.parametrize("permille", [0, 125, 500, 875, 1000])
+def test_adaptive_coverage_and_legality(permille):
+    q, k, cu, ms = _adaptive_case(seed=permille)
+    bm, bn, g = 4, 2, 2
+    r = oracle.route_adaptive(q, k, cu, ms, bm, bn, g, permille)
+    tm_ = -(-ms // bm)
+    assert r.shape == (len(cu) - 1, 2, tm_, 64)
+    for b in range(len(cu) - 1):
+        L = int(cu[b + 1] - cu[b])
+        for m in range(tm_):
+            if m * bm >= L:
+                assert not r[b, :, m].any()
+                continue
+            G = ((min((m + 1) * bm, L) - 1) // bn) // g + 1
+            assert not r[b, :, m, G:].any()
+            assert (r[b, :, m, :G].sum(axis=-1) ==
+                    (permille * G + 500) // 1000).all()
+
+
+def test_adaptive_head_map_regroups_query_heads():
+    q, k, cu, ms = _adaptive_case(seed=11)
+    # heads 0, 2 -> KV head 0 and 1, 3 -> KV head 1 through a map equals the
+    # contiguous grouping of the same heads reordered
+    a = oracle.route_adaptive(q, k, cu, ms, 4, 3, 1, 500)
+    b = oracle.route_adaptive(q[:, [0, 2, 1, 3]], k, cu, ms, 4, 3, 1, 500,
+                              head_map=[0, 1, 0, 1])
+    assert np.array_equal(a, b)
+
+
+def test_fp16_fixed_is_exact():
+    vals = np.array([0.0, -0.0, 2.0 ** -24, -(2.0 ** -24), 2.0 ** -14, 1.0,
+                     -1.5, 65504.0, 1.0009765625], np.float16)
+    want = [0, 0, 1, -1, 2 ** 10, 2 ** 24, -3 * 2 ** 23, 65504 * 2 ** 24,
+            2 ** 24 + 2 ** 14]
+    assert oracle.fp16_fixed(vals).tolist() == want
