@@ -101,6 +101,11 @@ def parse_args(argv=None):
     ap.add_argument("--quant-on-chip", action="store_true",
                     help="quantise Q and K tiles inside the attention kernel "
                          "(no separate quantiser launches)")
+    ap.add_argument("--routing", choices=["given", "adaptive"], default="given",
+                    help="given: the workload's routing bytes are an input and "
+                         "are packed each step; adaptive: each step derives "
+                         "the routing words from Q and K on the device at the "
+                         "workload's INT8 coverage")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args(argv)
@@ -361,17 +366,36 @@ def run_gpu(args):
         del k, v
         k = v = None
     on_chip = args.quant_on_chip and not kv8
-    launches_per_step = 2 if on_chip else (3 if kv8 else 4)
+    adaptive = args.routing == "adaptive"
+    if adaptive and kv8:
+        raise SystemExit("--routing adaptive needs fp16 K (not an INT8 KV cache)")
+    launches_per_step = (2 if on_chip else (3 if kv8 else 4)) + \
+        (1 if adaptive else 0)
+    permille = int(round(w.coverage * 1000))
+    ws = None
+    if adaptive:
+        ws = torch.empty(max(16, tm.tilemix_route_adaptive_workspace_bytes(
+            len(lens), ms, w.hkv, w.d, w.block_m)), dtype=torch.uint8,
+            device=dev)
 
-    def step(attn_events=None):
+    def step(attn_events=None, route_events=None):
         if not on_chip:
             tm.tilemix_quantize_blockwise(q, cu, ms, w.quant_block_q, x8=q8,
                                           scale=sq, status=status)
         if not kv8 and not on_chip:
             tm.tilemix_quantize_blockwise(k, cu, ms, w.quant_block_k, x8=k8,
                                           scale=sk, status=status)
-        tm.tilemix_pack_mask(route, cu, ms, w.block_m, w.block_n, g, mask=mask,
-                             status=status)
+        if route_events:
+            route_events[0].record(stream)
+        if adaptive:
+            tm.tilemix_route_adaptive(q, k, cu, ms, w.block_m, w.block_n, g,
+                                      permille, workspace=ws, mask=mask,
+                                      want_route=False, status=status)
+        else:
+            tm.tilemix_pack_mask(route, cu, ms, w.block_m, w.block_n, g,
+                                 mask=mask, status=status)
+        if route_events:
+            route_events[1].record(stream)
         if attn_events:
             attn_events[0].record(stream)
         tm.tilemix_attn_prefill(
@@ -390,7 +414,7 @@ def run_gpu(args):
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()} during warmup")
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)]
           for _ in range(args.steps)]
     smi_index = local
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
@@ -405,13 +429,14 @@ def run_gpu(args):
         for i in range(args.steps):
             flush.zero_()
             ev[i][0].record(stream)
-            step((ev[i][1], ev[i][2]))
+            step((ev[i][1], ev[i][2]), (ev[i][4], ev[i][5]))
             ev[i][3].record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     step_ms = [e[0].elapsed_time(e[3]) for e in ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    route_ms = [e[4].elapsed_time(e[5]) for e in ev]
     total_ms = max_over_ranks(sum(step_ms), dev)
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()} in timed region")
@@ -431,7 +456,10 @@ def run_gpu(args):
             cu_pin.numel() * 4
         d2h = out_h.numel() * out_h.element_size()
 
-        dev_of = {"q": q, "route": route}
+        if adaptive:   # the routing is derived on the device
+            h2d -= pin["route"].numel()
+            del pin["route"]
+        dev_of = {"q": q} if adaptive else {"q": q, "route": route}
         if kv8:
             dev_of.update(k8=k8, k_scale=sk, v8=v8, v_scale=sv)
         else:
@@ -490,6 +518,18 @@ def run_gpu(args):
             T, w.hq, w.hkv, w.d, wk["int8_pair_share"]),
     }
 
+    route_roof = None
+    if adaptive:
+        # the sums pass reads Q and K once; the words written are negligible
+        nbytes = T * (w.hq + w.hkv) * w.d * 2
+        r_s = statistics.mean(route_ms) * 1e-3
+        gbs = nbytes / r_s / 1e9
+        route_roof = {"bound": "hbm", "achieved": round(gbs, 1),
+                      "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                      "frac": round(gbs / float(peaks["hbm_gbs"]), 4),
+                      "bytes_per_launch": nbytes,
+                      "kernels": "sums_kernel + rank_kernel"}
+
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         rate, desc, cores = oracle_sample_rate(inp, args.cpu_seconds)
@@ -502,7 +542,12 @@ def run_gpu(args):
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp16+int8", "data": "synthetic",
         "config": dict(workload_config(w, inp, wk["int8_pair_share"]),
-                       quantisation="on chip" if on_chip else "quantise once"),
+                       quantisation="on chip" if on_chip else "quantise once",
+                       routing=("adaptive (on device, exact logit-sum "
+                                f"statistic, {permille} permille INT8)"
+                                if adaptive else "given routing bytes")),
+        "routing_ms": round(statistics.mean(route_ms), 4),
+        "routing_roofline": route_roof,
         "effective_tflops": wk["effective"] / (ms_step * 1e-3) / 1e12 * world,
         "attn_effective_tflops": achieved,
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,

@@ -179,6 +179,67 @@ tilemix_status tilemix_route_template(
     uint8_t* route, int32_t* status, tilemix_stream_t stream);
 
 /*
+ * Adaptive routing from a cheap score statistic, run on the device before
+ * the attention call.  Pages: paperlayer summary, Limitations (the kernel
+ * interface accepts static or adaptive routing policies) and appendix G.5
+ * (routing that keeps high-mass attention blocks in FP16 protects accuracy).
+ * The pages define no statistic; this library's reading:
+ *
+ * For query-tile row m of sequence b and KV head hk, with G legal groups,
+ *   Sq[c]   = sum over the row's in-sequence query rows i and the query
+ *             heads h of hk of X(q[i][h][c]),
+ *   Sk_j[c] = sum over the in-sequence keys of group j (key tiles
+ *             g*j .. g*j+g-1) of X(k[key][hk][c]),
+ *   I_j     = sum_c Sq[c] * Sk_j[c]  = 2^48 x the sum of all raw logits
+ *             q.k between the row's queries (over hk's heads) and the
+ *             group's keys,
+ * where X(v) = v * 2^24 is the exact integer value of an fp16 number; every
+ * sum is exact (64-bit for Sq, Sk; 128-bit for I), so the ranking does not
+ * depend on summation order.  k_int8 = (int8_permille * G + 500) / 1000; the
+ * G - k_int8 groups with the largest I_j stay FP16 (ties to the smaller j),
+ * the rest INT8.  Output: route bytes as tilemix_route_template, and / or
+ * the routing words the attention call reads.
+ *
+ *   q, k           dev fp16 [T, hq, d] / [T, hkv, d], 16-byte aligned;
+ *                  d a multiple of 8 in [8, 256]
+ *   head_map       optional dev int32 [hq] (NULL: contiguous groups of
+ *                  hq / hkv query heads)
+ *   workspace      dev scratch of at least
+ *                  tilemix_route_adaptive_workspace_bytes() bytes (8 * d *
+ *                  batch * hkv * (Tm_max + 64)), 16-byte aligned, owned by
+ *                  the caller; overwritten; must not be shared with another
+ *                  call that may run at the same time
+ *   route          optional dev uint8 [batch, hkv, Tm_max, 64], 16-byte
+ *                  aligned; bytes past a row's G legal groups and rows past
+ *                  a sequence's end are written 0
+ *   mask           optional dev uint64 [batch, hkv, Tm_max], 8-byte aligned:
+ *                  the same decisions as packed routing words, equal to
+ *                  tilemix_pack_mask of `route` (at least one of route and
+ *                  mask is given)
+ *
+ * Errors: INVALID_ARG for null or misaligned pointers, bad sizes, a
+ * permille outside [0, 1000], more than 64 groups or a short workspace;
+ * UNSUPPORTED for tiles so large that the exact integer arithmetic could
+ * overflow: with rows = block_m * query heads per KV head (hq with a
+ * head_map) and keys = g * block_n, it needs rows, keys < 2^15, rows * d and
+ * keys * d < 2^22, and rows * keys * d < 2^47.  Device side (status word): BAD_SEQLENS for
+ * cu_seqlens outside [0, total_tokens] or above max_seqlen, or a head_map
+ * entry outside [0, hkv); such a sequence's rows get no FP16 choice.
+ * Asynchronous on `stream`; allocates nothing.  The workspace query returns
+ * 0 for negative or zero sizes.
+ */
+size_t tilemix_route_adaptive_workspace_bytes(int batch, int max_seqlen,
+                                              int hkv, int head_dim,
+                                              int block_m);
+
+tilemix_status tilemix_route_adaptive(
+    const void* q, const void* k, const int32_t* cu_seqlens, int batch,
+    int max_seqlen, int total_tokens, int hq, int hkv, int head_dim,
+    const int32_t* head_map, int block_m, int block_n, int group,
+    int int8_permille, void* workspace, size_t workspace_bytes,
+    uint8_t* route, uint64_t* mask, int32_t* status, tilemix_stream_t stream);
+
+/*
  * Arguments of tilemix_attn_prefill.  Zero-initialise, set struct_size =
  * sizeof(tilemix_attn_params), then fill the fields.
  */

@@ -24,8 +24,9 @@ from pathlib import Path
 __all__ = [
     "TilemixError", "lib", "library_path", "EXPORTED_SYMBOLS",
     "tilemix_quantize_blockwise", "tilemix_pack_mask", "tilemix_attn_prefill",
-    "tilemix_route_template", "tilemix_status_string", "tilemix_last_error",
-    "tilemix_version", "KV_FP16", "KV_INT8", "FLAG_FP16_ONLY",
+    "tilemix_route_template", "tilemix_route_adaptive",
+    "tilemix_route_adaptive_workspace_bytes", "tilemix_status_string",
+    "tilemix_last_error", "tilemix_version", "KV_FP16", "KV_INT8", "FLAG_FP16_ONLY",
     "FLAG_QUANT_ON_CHIP", "STATUS",
     "LAYOUTS",
 ]
@@ -47,7 +48,8 @@ LAYOUTS = {"all_fp16": 0, "all_int8": 1, "band": 2, "global": 3,
 # Every function include/tilemix.h declares.
 EXPORTED_SYMBOLS = (
     "tilemix_quantize_blockwise", "tilemix_pack_mask", "tilemix_attn_prefill",
-    "tilemix_route_template", "tilemix_status_string", "tilemix_last_error",
+    "tilemix_route_template", "tilemix_route_adaptive_workspace_bytes",
+    "tilemix_route_adaptive", "tilemix_status_string", "tilemix_last_error",
     "tilemix_version",
 )
 
@@ -99,6 +101,12 @@ def _load() -> C.CDLL:
     lib.tilemix_route_template.restype = i32
     lib.tilemix_route_template.argtypes = [
         i32, i32, C.c_uint64, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+    lib.tilemix_route_adaptive_workspace_bytes.restype = C.c_size_t
+    lib.tilemix_route_adaptive_workspace_bytes.argtypes = [i32] * 5
+    lib.tilemix_route_adaptive.restype = i32
+    lib.tilemix_route_adaptive.argtypes = [
+        vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, i32, i32, i32, vp,
+        C.c_size_t, vp, vp, vp, vp]
     lib.tilemix_attn_prefill.restype = i32
     lib.tilemix_attn_prefill.argtypes = [C.POINTER(AttnParams), vp]
     lib.tilemix_status_string.restype = C.c_char_p
@@ -254,6 +262,55 @@ def tilemix_route_template(layout, int8_permille: int, cu_seqlens,
         max_seqlen, hkv, block_m, block_n, group, _ptr(route), _ptr(status),
         _stream(stream)), "tilemix_route_template")
     return route
+
+
+def tilemix_route_adaptive_workspace_bytes(batch: int, max_seqlen: int,
+                                           hkv: int, head_dim: int,
+                                           block_m: int) -> int:
+    """Bytes of device scratch tilemix_route_adaptive needs."""
+    return int(lib.tilemix_route_adaptive_workspace_bytes(
+        batch, max_seqlen, hkv, head_dim, block_m))
+
+
+def tilemix_route_adaptive(q, k, cu_seqlens, max_seqlen: int, block_m: int,
+                           block_n: int, group: int, int8_permille: int, *,
+                           head_map=None, workspace=None, route=None,
+                           mask=None, want_route: bool = True, status=None,
+                           stream=None):
+    """Route bytes [B, Hkv, ceil(max_seqlen/block_m), 64] (uint8, 1 = INT8)
+    chosen from the data: per query-tile row, the groups whose summed raw
+    logits with the row are largest stay FP16.  q fp16 [T, hq, d], k fp16
+    [T, hkv, d].  `workspace` (uint8 CUDA tensor) is allocated here when not
+    given.  Returns the route bytes, or (route, mask) when `mask` (uint64
+    words [B, Hkv, Tm], int64 CUDA tensor) is given; want_route=False skips
+    the bytes (route is then None)."""
+    torch = _torch()
+    _dev(q, "q", torch.float16)
+    _dev(k, "k", torch.float16)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    _dev(head_map, "head_map", torch.int32)
+    t, hq, d = q.shape
+    hkv = k.shape[1]
+    batch = cu_seqlens.numel() - 1
+    tm = -(-max_seqlen // block_m)
+    need = tilemix_route_adaptive_workspace_bytes(batch, max_seqlen, hkv, d,
+                                                  block_m)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8,
+                                device=q.device)
+    _dev(workspace, "workspace")
+    if route is None and want_route:
+        route = torch.empty((batch, hkv, tm, 64), dtype=torch.uint8,
+                            device=q.device)
+    _dev(route, "route", torch.uint8)
+    _dev(mask, "mask", torch.int64)
+    _check(lib.tilemix_route_adaptive(
+        _ptr(q), _ptr(k), _ptr(cu_seqlens), batch, max_seqlen, t, hq, hkv, d,
+        _ptr(head_map), block_m, block_n, group, int8_permille,
+        _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(route), _ptr(mask), _ptr(status), _stream(stream)),
+        "tilemix_route_adaptive")
+    return route if mask is None else (route, mask)
 
 
 def tilemix_attn_prefill(q, k, v, cu_seqlens, max_seqlen: int, *, q8=None,

@@ -40,6 +40,17 @@ cudaError_t launch_route_template(int layout, int permille, uint64_t seed,
                                   int block_n, int group, uint8_t* route,
                                   int32_t* status, cudaStream_t stream);
 
+size_t route_adaptive_workspace(int batch, int max_seqlen, int hkv, int d,
+                                int block_m);
+cudaError_t launch_route_adaptive(const void* q, const void* k,
+                                  const int32_t* cu_seqlens, int batch,
+                                  int max_seqlen, int total_tokens, int hq,
+                                  int hkv, int d, const int32_t* head_map,
+                                  int block_m, int block_n, int group,
+                                  int permille, void* workspace, uint8_t* route,
+                                  uint64_t* mask, int32_t* status,
+                                  cudaStream_t stream);
+
 // Everything the fused attention kernel reads.  Passed by value as a
 // __grid_constant__ parameter; the tensor maps must stay 64-byte aligned.
 struct AttnParams {

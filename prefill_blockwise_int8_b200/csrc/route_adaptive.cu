@@ -1,0 +1,302 @@
+// Adaptive routing from exact block logit sums, for sm_100a.
+//
+// Method: TileMix (arXiv 2608.17336), paperlayer summary Limitations (the
+// kernel interface consumes static or adaptive routing policies) and
+// appendix G.5 (routing that keeps high-mass attention blocks in FP16).  The
+// statistic is this library's reading (stated with the C declaration): the
+// sum of all raw logits between a query-tile row and a key group, computed
+// exactly as (sum of the row's queries) . (sum of the group's keys) with
+// fp16 values scaled to exact integers, so the result and the ranking do not
+// depend on the order of any sum.
+//
+// Pass 1 (sums_kernel): one CTA per (query tile, or run of key groups of
+// about 256 keys; KV head; sequence); each thread reads 16-byte chunks of
+// rows (coalesced across the CTA) and keeps eight exact channel sums
+// (rescaled doubles for runs, then int64); the CTA adds the slices' totals
+// through shared memory.  Q and K are each read once.
+// Pass 2 (rank_kernel): one CTA per (sequence, KV head, query-tile row);
+// thread j forms the dot product of the row's sums with group j's in 24-bit
+// limbs, ranks group j, writes its route byte, and warp ballots give the
+// packed routing word.
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+namespace tilemix {
+namespace {
+
+constexpr int kGroups = 64;
+constexpr int kSumThreads = 128;
+
+// Exact sums of fp16 values in doubles, without a conversion instruction.
+//
+// Placing the 15 magnitude bits of an fp16 value (5 exponent, 10 mantissa)
+// at the top of a double's exponent and mantissa fields, with the sign bit
+// moved along, gives exactly the value times 2^-1008: an exponent field e
+// reads as 2^(e - 1023) (1 + m / 1024) = 2^-1008 * 2^(e - 15) (1 + m / 1024),
+// and e = 0 reads as the subnormal 2^-1022 m / 2^52 * 2^42 = 2^-1008 m 2^-24.
+// Every such value is a multiple of 2^-1032 below 2^-992 in magnitude, so a
+// double sum of at most 2^13 of them is a multiple of 2^-1032 below 2^-979:
+// it needs at most 53 significant bits and every addition is exact
+// (subnormal doubles are kept; nothing here flushes them).  Runs of at most
+// kExactRun rows are summed so and moved, times 2^1032 (exact), into int64
+// totals of value * 2^24.  (An Inf or NaN input gives an unspecified
+// ranking.)
+constexpr int kExactRun = 4096;
+
+__device__ __forceinline__ double scaled_lo(uint32_t w) {
+  const uint32_t hi = ((w & 0x7fffu) << 10) | ((w << 16) & 0x80000000u);
+  return __hiloint2double(static_cast<int>(hi), 0);
+}
+
+__device__ __forceinline__ double scaled_hi(uint32_t w) {
+  const uint32_t hi = ((w >> 6) & 0x01fffc00u) | (w & 0x80000000u);
+  return __hiloint2double(static_cast<int>(hi), 0);
+}
+
+__device__ __forceinline__ void add_chunk(double (&a)[8], uint4 w) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    a[2 * i] += scaled_lo(u[i]);
+    a[2 * i + 1] += scaled_hi(u[i]);
+  }
+}
+
+// Running exact sums of one thread's eight channels: doubles for runs of at
+// most kExactRun rows, then int64 totals of value * 2^24.
+struct ExactSums {
+  double a[8];
+  int64_t t[8];
+  int run;
+
+  __device__ __forceinline__ void clear() {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      a[e] = 0.0;
+      t[e] = 0;
+    }
+    run = 0;
+  }
+  __device__ __forceinline__ void settle() {
+    // 2^1032 in two exact power-of-two steps (2^1032 is not a double)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      t[e] += __double2ll_rn(a[e] * 0x1p1000 * 0x1p32);
+      a[e] = 0.0;
+    }
+    run = 0;
+  }
+  // rows first, first + step, ... < last of a [rows, stride] fp16 matrix,
+  // 16-byte chunk at `base`
+  __device__ __forceinline__ void add_rows(const uint16_t* __restrict__ base,
+                                           size_t stride, int first, int last,
+                                           int step) {
+    const uint16_t* p = base + static_cast<size_t>(first) * stride;
+    const size_t dp = static_cast<size_t>(step) * stride;
+#pragma unroll 4
+    for (int i = first; i < last; i += step, p += dp) {
+      add_chunk(a, __ldg(reinterpret_cast<const uint4*>(p)));
+      if (++run == kExactRun) settle();
+    }
+  }
+};
+
+// The CTA's slices hold totals for the same channels; add them in order.
+__device__ __forceinline__ void reduce_slices(const ExactSums& s,
+                                              int64_t* part_s, int rs, int cc,
+                                              int slices, int d,
+                                              int64_t* __restrict__ out) {
+  if (rs < slices) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part_s[rs * d + cc * 8 + e] = s.t[e];
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < d; c += kSumThreads) {
+    int64_t total = 0;
+    for (int r = 0; r < slices; ++r) total += part_s[r * d + c];
+    out[c] = total;
+  }
+  __syncthreads();
+}
+
+// blockIdx.x < tm: query tile u (its rows over the KV head's query heads);
+// otherwise key groups gpc * (x - tm) .. + gpc - 1 (groups past 63 skipped).
+__global__ void __launch_bounds__(kSumThreads)
+    sums_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                const int32_t* __restrict__ cu_seqlens,
+                const int32_t* __restrict__ head_map, int max_seqlen,
+                int total_tokens, int hq, int hkv, int d, int tm, int block_m,
+                int keys_per_group, int gpc, int64_t* __restrict__ sq,
+                int64_t* __restrict__ sk, int32_t* status) {
+  // per-slice channel totals: slices * d = 8 * kSumThreads entries
+  __shared__ int64_t part_s[8 * kSumThreads];
+  const int u = blockIdx.x;
+  const int hk = blockIdx.y;
+  const int b = blockIdx.z;
+  const int chunks = d >> 3;
+  const int slices = kSumThreads / chunks;
+  const int cc = threadIdx.x % chunks;
+  const int rs = threadIdx.x / chunks;
+  const int start = cu_seqlens[b];
+  const int len = cu_seqlens[b + 1] - start;
+  const bool valid = start >= 0 && len >= 0 && len <= max_seqlen &&
+                     start + len <= total_tokens;
+  if (!valid && threadIdx.x == 0 && u == 0 && hk == 0)
+    report_status(status, kStatusBadSeqlens);
+  const bool active = valid && rs < slices;
+  ExactSums s;
+  s.clear();
+  if (u < tm) {
+    if (active) {
+      const int r0 = u * block_m + rs, r1 = min((u + 1) * block_m, len);
+      const size_t stride = static_cast<size_t>(hq) * d;
+      const uint16_t* base = q + static_cast<size_t>(start) * stride + cc * 8;
+      if (head_map) {
+        for (int h = 0; h < hq; ++h) {
+          const int hm = head_map[h];
+          if (hm < 0 || hm >= hkv) {
+            if (threadIdx.x == 0) report_status(status, kStatusBadSeqlens);
+          } else if (hm == hk) {
+            s.add_rows(base + static_cast<size_t>(h) * d, stride, r0, r1, slices);
+          }
+        }
+      } else {
+        const int per = hq / hkv;  // hkv divides hq without a map
+        for (int h = hk * per; h < (hk + 1) * per; ++h)
+          s.add_rows(base + static_cast<size_t>(h) * d, stride, r0, r1, slices);
+      }
+    }
+    s.settle();
+    reduce_slices(s, part_s, rs, cc, slices, d,
+                  sq + ((static_cast<size_t>(b) * hkv + hk) * tm + u) * d);
+  } else {
+    const size_t stride = static_cast<size_t>(hkv) * d;
+    const uint16_t* base =
+        k + static_cast<size_t>(start) * stride + static_cast<size_t>(hk) * d + cc * 8;
+    const int j0 = (u - tm) * gpc;
+    for (int j = j0; j < min(j0 + gpc, kGroups); ++j) {
+      if (active)
+        s.add_rows(base, stride, j * keys_per_group + rs,
+                   min((j + 1) * keys_per_group, len), slices);
+      s.settle();
+      reduce_slices(s, part_s, rs, cc, slices, d,
+                    sk + ((static_cast<size_t>(b) * hkv + hk) * kGroups + j) * d);
+      s.clear();
+    }
+  }
+}
+
+// One CTA of 64 threads per (sequence, KV head, query-tile row); thread j
+// computes the statistic of group j over all channels in 24-bit limbs:
+// with Sq = a1 * 2^24 + a0 and Sk = b1 * 2^24 + b0 (0 <= a0, b0 < 2^24),
+//   Sq . Sk = 2^48 sum a1 b1 + 2^24 sum (a0 b1 + a1 b0) + sum a0 b0.
+// The host admits only tiles with rows, keys < 2^15, rows * d and keys * d
+// < 2^22 and rows * keys * d < 2^47 (rows = query rows of a tile times its
+// query heads, keys = keys of a group), where |Sq| < 2^40 rows and |Sk| <
+// 2^40 keys: the limbs fit int32, the three low sums int64 (their sum
+// included), and the statistic int128.  Thread j then ranks group j, writes
+// its byte, and warp ballots give the routing word.
+__global__ void __launch_bounds__(64)
+    rank_kernel(const int32_t* __restrict__ cu_seqlens, int max_seqlen,
+                int total_tokens, int hkv, int tm, int d, int block_m,
+                int block_n, int group, int permille,
+                const int64_t* __restrict__ sq, const int64_t* __restrict__ sk,
+                uint8_t* __restrict__ route, uint64_t* __restrict__ mask) {
+  __shared__ int2 q_s[256];  // (a0, a1) per channel
+  __shared__ __int128 imp_s[kGroups];
+  const int j = threadIdx.x;
+  const int lane = j & 31;
+  const long long row = blockIdx.x;  // (b * hkv + hk) * tm + m
+  const int m = static_cast<int>(row % tm);
+  const long long bh = row / tm;
+  const int b = static_cast<int>(bh / hkv);
+  const int start = cu_seqlens[b];
+  const int len = cu_seqlens[b + 1] - start;
+  int G = 0;  // an invalid sequence was reported by the first pass
+  if (start >= 0 && len >= 0 && len <= max_seqlen &&
+      start + len <= total_tokens && static_cast<long long>(m) * block_m < len)
+    G = ((min((m + 1) * block_m, len) - 1) / block_n) / group + 1;
+  for (int c = j; c < d; c += 64) {
+    const int64_t v = sq[row * d + c];
+    q_s[c] = make_int2(static_cast<int>(v & 0xFFFFFF), static_cast<int>(v >> 24));
+  }
+  __syncthreads();
+  if (j < G) {
+    const longlong2* kg =
+        reinterpret_cast<const longlong2*>(sk + (bh * kGroups + j) * d);
+    int64_t lo = 0, mid = 0;
+    __int128 hi = 0;
+#pragma unroll 4
+    for (int c2 = 0; c2 < (d >> 1); ++c2) {
+      const longlong2 kv = __ldg(kg + c2);
+      const int64_t kk[2] = {kv.x, kv.y};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int2 a = q_s[2 * c2 + e];
+        const int b0 = static_cast<int>(kk[e] & 0xFFFFFF);
+        const int b1 = static_cast<int>(kk[e] >> 24);
+        lo += static_cast<int64_t>(a.x) * b0;
+        mid += static_cast<int64_t>(a.x) * b1 + static_cast<int64_t>(a.y) * b0;
+        hi += static_cast<int64_t>(a.y) * b1;
+      }
+    }
+    imp_s[j] = (hi << 48) + (static_cast<__int128>(mid) << 24) + lo;
+  }
+  __syncthreads();
+  const int k_fp16 = G - (permille * G + 500) / 1000;
+  uint8_t bit = 0;
+  if (j < G) {
+    const __int128 v = imp_s[j];
+    int rank = 0;  // groups ahead of j: a larger statistic, or equal and smaller index
+    for (int i = 0; i < G; ++i) {
+      const __int128 x = imp_s[i];
+      rank += (x > v || (x == v && i < j)) ? 1 : 0;
+    }
+    bit = rank >= k_fp16 ? 1 : 0;
+  }
+  if (route) route[row * 64 + j] = bit;
+  const uint32_t half = __ballot_sync(0xffffffffu, bit != 0);
+  if (mask && lane == 0) reinterpret_cast<uint32_t*>(mask + row)[j >> 5] = half;
+}
+
+}  // namespace
+
+size_t route_adaptive_workspace(int batch, int max_seqlen, int hkv, int d,
+                                int block_m) {
+  const size_t tm = (static_cast<size_t>(max_seqlen) + block_m - 1) / block_m;
+  return sizeof(int64_t) * d * static_cast<size_t>(batch) * hkv *
+         (tm + kGroups);
+}
+
+cudaError_t launch_route_adaptive(const void* q, const void* k,
+                                  const int32_t* cu_seqlens, int batch,
+                                  int max_seqlen, int total_tokens, int hq,
+                                  int hkv, int d,
+                                  const int32_t* head_map, int block_m,
+                                  int block_n, int group, int permille,
+                                  void* workspace, uint8_t* route,
+                                  uint64_t* mask, int32_t* status,
+                                  cudaStream_t stream) {
+  const int tm = (max_seqlen + block_m - 1) / block_m;
+  int64_t* sq = static_cast<int64_t*>(workspace);
+  int64_t* sk = sq + static_cast<size_t>(d) * batch * hkv * tm;
+  // key CTAs take gpc consecutive groups, about 256 keys in all
+  const int kpg = group * block_n;
+  const int gpc = kpg >= 256 ? 1 : 256 / kpg;
+  const dim3 g1(tm + (kGroups + gpc - 1) / gpc, hkv, batch);
+  sums_kernel<<<g1, kSumThreads, 0, stream>>>(
+      static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+      cu_seqlens, head_map, max_seqlen, total_tokens, hq, hkv, d, tm, block_m,
+      kpg, gpc, sq, sk, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long rows = static_cast<long long>(batch) * hkv * tm;
+  rank_kernel<<<static_cast<unsigned>(rows), 64, 0, stream>>>(
+      cu_seqlens, max_seqlen, total_tokens, hkv, tm, d, block_m, block_n, group,
+      permille, sq, sk, route, mask);
+  return cudaGetLastError();
+}
+
+}  // namespace tilemix

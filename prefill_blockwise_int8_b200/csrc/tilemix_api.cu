@@ -214,6 +214,82 @@ tilemix_status tilemix_route_template(int layout, int int8_permille,
   return ok();
 }
 
+size_t tilemix_route_adaptive_workspace_bytes(int batch, int max_seqlen,
+                                              int hkv, int head_dim,
+                                              int block_m) {
+  if (batch < 0 || max_seqlen < 0 || hkv <= 0 || head_dim <= 0 || block_m <= 0)
+    return 0;
+  return tilemix::route_adaptive_workspace(batch, max_seqlen, hkv, head_dim,
+                                           block_m);
+}
+
+tilemix_status tilemix_route_adaptive(
+    const void* q, const void* k, const int32_t* cu_seqlens, int batch,
+    int max_seqlen, int total_tokens, int hq, int hkv, int head_dim,
+    const int32_t* head_map, int block_m, int block_n, int group,
+    int int8_permille, void* workspace, size_t workspace_bytes,
+    uint8_t* route, uint64_t* mask, int32_t* status, tilemix_stream_t stream) {
+  if (!q || !k || !cu_seqlens || (!route && !mask))
+    return fail(TILEMIX_ERR_INVALID_ARG, "route_adaptive: null pointer");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(route, 16) ||
+      !aligned(mask, 8) ||
+      !aligned(cu_seqlens, 4) || (head_map && !aligned(head_map, 4)) ||
+      (workspace && !aligned(workspace, 16)) || (status && !aligned(status, 4)))
+    return fail(TILEMIX_ERR_INVALID_ARG, "route_adaptive: misaligned pointer");
+  if (int8_permille < 0 || int8_permille > 1000)
+    return fail(TILEMIX_ERR_INVALID_ARG,
+                "route_adaptive: int8_permille %d not in [0, 1000]",
+                int8_permille);
+  if (batch < 0 || max_seqlen < 0 || total_tokens < 0 || hq <= 0 || hkv <= 0 ||
+      block_m <= 0 || block_n <= 0 || group <= 0)
+    return fail(TILEMIX_ERR_INVALID_ARG, "route_adaptive: bad size");
+  if (head_dim < 8 || head_dim > 256 || head_dim % 8 != 0)
+    return fail(TILEMIX_ERR_UNSUPPORTED,
+                "route_adaptive: head_dim %d not a multiple of 8 in [8, 256]",
+                head_dim);
+  if (!head_map && hq % hkv != 0)
+    return fail(TILEMIX_ERR_INVALID_ARG,
+                "route_adaptive: hq %d not a multiple of hkv %d and no head_map",
+                hq, hkv);
+  if (hkv > 65535 || batch > 65535)
+    return fail(TILEMIX_ERR_UNSUPPORTED, "route_adaptive: hkv or batch > 65535");
+  if (batch == 0 || max_seqlen == 0) return ok();
+  const long long tn = (static_cast<long long>(max_seqlen) + block_n - 1) / block_n;
+  if ((tn + group - 1) / group > 64)
+    return fail(TILEMIX_ERR_INVALID_ARG,
+                "route_adaptive: ceil(%lld key tiles / g=%d) > 64 routing bits",
+                tn, group);
+  // |fp16 * 2^24| < 2^40, so a tile's query sums stay below 2^40 * rows and
+  // a group's key sums below 2^40 * keys; the device's 24-bit limb products
+  // and the int128 statistic stay exact within these bounds.
+  const long long rows = static_cast<long long>(block_m) * (head_map ? hq : hq / hkv);
+  const long long keys = static_cast<long long>(group) * block_n;
+  if (rows >= (1ll << 15) || keys >= (1ll << 15) ||
+      rows * head_dim >= (1ll << 22) || keys * head_dim >= (1ll << 22) ||
+      rows * keys * head_dim >= (1ll << 47))
+    return fail(TILEMIX_ERR_UNSUPPORTED,
+                "route_adaptive: tile sizes too large for exact statistics");
+  const long long tm = (static_cast<long long>(max_seqlen) + block_m - 1) / block_m;
+  if (static_cast<long long>(batch) * hkv * tm > 0x7fffffffll)
+    return fail(TILEMIX_ERR_UNSUPPORTED, "route_adaptive: too many routing rows");
+  const size_t need = tilemix::route_adaptive_workspace(batch, max_seqlen, hkv,
+                                                        head_dim, block_m);
+  if (!workspace || workspace_bytes < need)
+    return fail(TILEMIX_ERR_INVALID_ARG,
+                "route_adaptive: workspace of %zu bytes, %zu needed",
+                workspace ? workspace_bytes : static_cast<size_t>(0), need);
+  tilemix_status d = check_device();
+  if (d != TILEMIX_OK) return d;
+  cudaError_t e = tilemix::launch_route_adaptive(
+      q, k, cu_seqlens, batch, max_seqlen, total_tokens, hq, hkv, head_dim,
+      head_map, block_m, block_n, group, int8_permille, workspace, route,
+      mask, status, stream);
+  if (e != cudaSuccess)
+    return fail(TILEMIX_ERR_CUDA, "route_adaptive launch: %s",
+                cudaGetErrorString(e));
+  return ok();
+}
+
 tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
                                     tilemix_stream_t stream) {
   if (!a) return fail(TILEMIX_ERR_INVALID_ARG, "attn: params is NULL");

@@ -18,6 +18,27 @@ OK, INVALID, UNSUPPORTED, NO_DEVICE = 0, 1, 2, 6
 FAKE = 0x10000  # 64 KiB: 16-byte aligned, never dereferenced on the host
 
 
+def _device_visible():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:  # no torch: no device either
+        return False
+
+
+# A call that passes every host check would launch a kernel on the fake
+# pointers, so it is only made where no device exists (it then stops at the
+# device check); a reject stops before any launch and runs everywhere.
+DEVICE_VISIBLE = _device_visible()
+
+
+def accepted(fn, *args):
+    if DEVICE_VISIBLE:
+        return True
+    rc = fn(*args)
+    return rc in (NO_DEVICE, OK)
+
+
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
@@ -87,8 +108,7 @@ def call(p):
 def test_attn_host_checks_accept_a_valid_call():
     # valid arguments get past every host check; with no GPU in this
     # process the call then stops at the device check
-    rc = call(good_params())
-    assert rc in (NO_DEVICE, OK), tm.tilemix_last_error()
+    assert accepted(call, good_params()), tm.tilemix_last_error()
 
 
 @pytest.mark.parametrize("field,value,expect", [
@@ -119,12 +139,12 @@ def test_attn_block_m64_needs_block_n64():
 def test_attn_fp16_only_needs_no_int8_operands():
     p = good_params(flags=tm.FLAG_FP16_ONLY, mask=0, q8=0, k8=0, q_scale=0,
                     k_scale=0)
-    assert call(p) in (NO_DEVICE, OK)
+    assert accepted(call, p)
 
 
 def test_group_lifts_the_64_bit_limit():
     p = good_params(max_seqlen=64 * 64 * 2, total_tokens=64 * 64 * 4, group=2)
-    assert call(p) in (NO_DEVICE, OK)
+    assert accepted(call, p)
 
 
 def test_quantize_and_pack_host_checks():
@@ -133,11 +153,11 @@ def test_quantize_and_pack_host_checks():
     assert q(FAKE, FAKE, 1, 128, 128, 2, 60, 128, FAKE, FAKE, None, None) == INVALID
     assert q(FAKE, FAKE, 1, 128, 128, 2, 256, 256, FAKE, FAKE, None, None) == INVALID
     assert q(FAKE + 4, FAKE, 1, 128, 128, 2, 64, 128, FAKE, FAKE, None, None) == INVALID
-    assert q(FAKE, FAKE, 1, 128, 128, 2, 64, 128, FAKE, FAKE, None, None) in (NO_DEVICE, OK)
+    assert accepted(q, FAKE, FAKE, 1, 128, 128, 2, 64, 128, FAKE, FAKE, None, None)
     assert q(FAKE, FAKE, 0, 0, 0, 2, 64, 128, FAKE, FAKE, None, None) == OK
     pk = tm.lib.tilemix_pack_mask
     assert pk(FAKE, FAKE, 1, 64 * 65, 1, 64, 64, 1, FAKE, None, None) == INVALID
-    assert pk(FAKE, FAKE, 1, 64 * 65, 1, 64, 64, 2, FAKE, None, None) in (NO_DEVICE, OK)
+    assert accepted(pk, FAKE, FAKE, 1, 64 * 65, 1, 64, 64, 2, FAKE, None, None)
     assert pk(FAKE + 8, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
     assert pk(None, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
 
@@ -145,7 +165,7 @@ def test_quantize_and_pack_host_checks():
 def test_route_template_host_checks():
     rt = tm.lib.tilemix_route_template
     # layout, int8_permille, seed, cu, batch, max_seqlen, hkv, bm, bn, g, route
-    assert rt(2, 750, 1, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) in (NO_DEVICE, OK)
+    assert accepted(rt, 2, 750, 1, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None)
     assert rt(8, 750, 1, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
     assert rt(-1, 750, 1, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
     assert rt(2, 1001, 1, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
@@ -154,3 +174,34 @@ def test_route_template_host_checks():
     assert rt(2, 750, 1, FAKE, 1, 128, 1, 64, 64, 1, FAKE + 8, None, None) == INVALID
     assert rt(2, 750, 1, None, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
     assert rt(2, 750, 1, FAKE, 0, 0, 1, 64, 64, 1, FAKE, None, None) == OK
+
+
+def test_route_adaptive_host_checks():
+    ra = tm.lib.tilemix_route_adaptive
+    ws = tm.tilemix_route_adaptive_workspace_bytes(1, 128, 2, 128, 64)
+    assert ws == 8 * 128 * 1 * 2 * (2 + 64)
+    assert tm.tilemix_route_adaptive_workspace_bytes(-1, 128, 2, 128, 64) == 0
+
+    def args(**kw):
+        a = dict(q=FAKE, k=FAKE, cu=FAKE, batch=1, max_seqlen=128,
+                 total_tokens=128, hq=4, hkv=2, d=128, head_map=None, bm=64,
+                 bn=64, g=1, permille=750, ws=FAKE, ws_bytes=ws, route=FAKE,
+                 mask=None, status=None, stream=None)
+        a.update(kw)
+        return list(a.values())
+
+    assert accepted(ra, *args())
+    assert accepted(ra, *args(route=None, mask=FAKE))
+    assert ra(*args(ws_bytes=ws - 1)) == INVALID
+    assert ra(*args(ws=None)) == INVALID
+    assert ra(*args(route=None, mask=None)) == INVALID
+    assert ra(*args(mask=FAKE + 4)) == INVALID
+    assert ra(*args(q=FAKE + 8)) == INVALID
+    assert ra(*args(permille=1001)) == INVALID
+    assert ra(*args(hkv=3)) == INVALID            # 4 % 3 and no head_map
+    assert ra(*args(max_seqlen=64 * 65)) == INVALID
+    assert ra(*args(d=60)) == UNSUPPORTED
+    assert ra(*args(d=264)) == UNSUPPORTED
+    assert ra(*args(bn=1 << 15)) == UNSUPPORTED    # limbs could leave int32
+    assert ra(*args(hq=512, hkv=2, bm=128)) == UNSUPPORTED   # rows * d >= 2^22
+    assert ra(*args(batch=0, max_seqlen=0, ws=None, ws_bytes=0)) == OK

@@ -345,6 +345,111 @@ def test_route_template_through_attention(tm):
 
 
 # ----------------------------------------------------------------------------
+# adaptive routing: route bytes and routing words byte-exact against the
+# oracle's exact-integer statistic, then through attention
+# ----------------------------------------------------------------------------
+
+ADAPTIVE_CASES = {
+    # lens, hq, hkv, d, block_m, block_n, g, head_map, value recipe
+    "ragged_d128_bn64": ([700, 300, 1, 0, 1500], 4, 2, 128, 128, 64, 1, None, "outliers"),
+    "d64_bm64_g2": ([1000, 77], 6, 2, 64, 64, 64, 2, None, "normal"),
+    "d96_head_map": ([513], 6, 2, 96, 128, 128, 1, [1, 0, 0, 1, 1, 0], "normal"),
+    "ties_small_ints": ([640, 130], 2, 1, 32, 64, 64, 1, None, "ternary"),
+    "g5_long": ([20000], 2, 1, 64, 128, 64, 5, None, "normal"),
+    # a KV head no query head maps to: all statistics 0, ties everywhere
+    "head_map_idle_kv_head": ([300, 129], 2, 3, 64, 64, 64, 1, [2, 0], "normal"),
+}
+
+
+def adaptive_inputs(lens, hq, hkv, d, recipe, seed=21):
+    rng = np.random.default_rng(seed)
+    T = int(sum(lens))
+    if recipe == "ternary":   # many exactly equal statistics: tie-breaking
+        q = rng.integers(0, 2, (T, hq, d)).astype(np.float16)
+        k = rng.integers(-1, 2, (T, hkv, d)).astype(np.float16)
+        k[:, :, 1:] = 0
+    else:
+        q = rng.standard_normal((T, hq, d)).astype(np.float16)
+        k = rng.standard_normal((T, hkv, d)).astype(np.float16)
+        if recipe == "outliers":
+            q[:, :, 5] *= 40
+            k[:, :, 5] *= 40
+    return q, k
+
+
+@pytest.mark.parametrize("name", sorted(ADAPTIVE_CASES))
+def test_route_adaptive_bitexact(tm, name):
+    lens, hq, hkv, d, bm, bn, g, hmap, recipe = ADAPTIVE_CASES[name]
+    lens = np.array(lens, np.int32)
+    cu = W.cu_seqlens(lens)
+    ms = int(max(lens.max(), 1))
+    q, k = adaptive_inputs(lens, hq, hkv, d, recipe)
+    qd, kd, cud = dev_tensor(q), dev_tensor(k), dev_tensor(cu)
+    hm = None if hmap is None else dev_tensor(np.array(hmap, np.int32))
+    tmr = -(-ms // bm)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for permille in (0, 250, 750, 1000):
+        mask = torch.full((len(lens), hkv, tmr), -1, dtype=torch.int64,
+                          device="cuda")
+        route, mask = tm.tilemix_route_adaptive(
+            qd, kd, cud, ms, bm, bn, g, permille, head_map=hm, mask=mask,
+            status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        ref = oracle.route_adaptive(q, k, cu, ms, bm, bn, g, permille,
+                                    head_map=hmap)
+        assert np.array_equal(route.cpu().numpy(), ref), permille
+        words = oracle.pack_mask(ref, cu, ms, bm, bn, g)
+        assert np.array_equal(mask.cpu().numpy().view(np.uint64), words)
+
+
+def test_route_adaptive_full_size_sampled(tm):
+    # LLaMA-3.2-3B prefill shape: 8 x 4096 tokens, 24 / 8 heads, d 128,
+    # 128 x 64 tiles; the oracle checks two whole sequences
+    lens = np.full(8, 4096, np.int32)
+    cu = W.cu_seqlens(lens)
+    q, k = adaptive_inputs(lens, 24, 8, 128, "outliers", seed=4)
+    route = tm.tilemix_route_adaptive(dev_tensor(q), dev_tensor(k),
+                                      dev_tensor(cu), 4096, 128, 64, 1, 750)
+    torch.cuda.synchronize()
+    got = route.cpu().numpy()
+    for b in (0, 7):
+        sl = slice(int(cu[b]), int(cu[b + 1]))
+        ref = oracle.route_adaptive(q[sl], k[sl], np.array([0, 4096], np.int32),
+                                    4096, 128, 64, 1, 750)
+        assert np.array_equal(got[b], ref[0]), b
+
+
+def test_route_adaptive_bad_seqlens_reported(tm):
+    q, k = adaptive_inputs([100], 2, 1, 64, "normal")
+    cu = np.array([0, 100], np.int32)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    # a sequence longer than max_seqlen: reported, its rows route nothing
+    route = tm.tilemix_route_adaptive(dev_tensor(q), dev_tensor(k),
+                                      dev_tensor(cu), 64, 64, 64, 1, 500,
+                                      status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 5     # TILEMIX_ERR_BAD_SEQLENS
+    assert not route.cpu().numpy().any()
+
+
+def test_route_adaptive_through_attention(tm):
+    inp = small([900, 333], bn=64)
+    w = inp["workload"]
+    route = tm.tilemix_route_adaptive(
+        dev_tensor(inp["q"]), dev_tensor(inp["k"]), dev_tensor(inp["cu_seqlens"]),
+        inp["max_seqlen"], w.block_m, w.block_n, inp["group"], 750).cpu().numpy()
+    ref_route = oracle.route_adaptive(inp["q"], inp["k"], inp["cu_seqlens"],
+                                      inp["max_seqlen"], w.block_m, w.block_n,
+                                      inp["group"], 750)
+    assert np.array_equal(route, ref_route)
+    got = run_gpu(inp, route=route)
+    assert got["status"] == 0
+    ref, _ = run_oracle(inp, route=route)
+    compare(got["out"], ref)
+
+
+# ----------------------------------------------------------------------------
 # on-chip quantisation: identical to quantise-once, element for element
 # ----------------------------------------------------------------------------
 
