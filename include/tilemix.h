@@ -240,6 +240,35 @@ tilemix_status tilemix_route_adaptive(
     uint8_t* route, uint64_t* mask, int32_t* status, tilemix_stream_t stream);
 
 /*
+ * tilemix_route_adaptive without a caller workspace: the same checks, the
+ * same kernels and the same output, with the scratch taken from one static
+ * device array of TILEMIX_ROUTE_ADAPTIVE_STATIC_BYTES per device (reserved
+ * when the library's module loads on that device; this call allocates
+ * nothing, so it may be captured in a CUDA graph).  No counterpart in the
+ * TileMix pages: an interface convenience of this library.
+ *
+ * Errors: as tilemix_route_adaptive, and INVALID_ARG when the call would
+ * need more than TILEMIX_ROUTE_ADAPTIVE_STATIC_BYTES of scratch
+ * (tilemix_route_adaptive_workspace_bytes() says how much).
+ *
+ * Races: every call on a device shares the one scratch array.  Two calls
+ * whose work can overlap on the device (different streams without an event
+ * between them, different host threads, concurrent graph replays) overwrite
+ * each other's statistics and may write wrong routing without any error.
+ * Order such calls on one stream or with events; calls in one stream are
+ * safe.
+ */
+#define TILEMIX_ROUTE_ADAPTIVE_STATIC_BYTES (32u << 20)
+
+tilemix_status tilemix_route_adaptive_noalloc(
+    const void* q, const void* k, const int32_t* cu_seqlens, int batch,
+    int max_seqlen, int total_tokens, int hq, int hkv, int head_dim,
+    const int32_t* head_map, int block_m, int block_n, int group,
+    int int8_permille, uint8_t* route, uint64_t* mask, int32_t* status,
+    tilemix_stream_t stream);
+
+
+/*
  * Arguments of tilemix_attn_prefill.  Zero-initialise, set struct_size =
  * sizeof(tilemix_attn_params), then fill the fields.
  */

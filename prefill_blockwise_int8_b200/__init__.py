@@ -25,7 +25,8 @@ __all__ = [
     "TilemixError", "lib", "library_path", "EXPORTED_SYMBOLS",
     "tilemix_quantize_blockwise", "tilemix_pack_mask", "tilemix_attn_prefill",
     "tilemix_route_template", "tilemix_route_adaptive",
-    "tilemix_route_adaptive_workspace_bytes", "tilemix_status_string",
+    "tilemix_route_adaptive_workspace_bytes", "tilemix_route_adaptive_noalloc",
+    "ROUTE_ADAPTIVE_STATIC_BYTES", "tilemix_status_string",
     "tilemix_last_error", "tilemix_version", "KV_FP16", "KV_INT8", "FLAG_FP16_ONLY",
     "FLAG_QUANT_ON_CHIP", "STATUS",
     "LAYOUTS",
@@ -49,9 +50,13 @@ LAYOUTS = {"all_fp16": 0, "all_int8": 1, "band": 2, "global": 3,
 EXPORTED_SYMBOLS = (
     "tilemix_quantize_blockwise", "tilemix_pack_mask", "tilemix_attn_prefill",
     "tilemix_route_template", "tilemix_route_adaptive_workspace_bytes",
-    "tilemix_route_adaptive", "tilemix_status_string", "tilemix_last_error",
-    "tilemix_version",
+    "tilemix_route_adaptive", "tilemix_route_adaptive_noalloc",
+    "tilemix_status_string", "tilemix_last_error", "tilemix_version",
 )
+
+# TILEMIX_ROUTE_ADAPTIVE_STATIC_BYTES: the static scratch of
+# tilemix_route_adaptive_noalloc on each device.
+ROUTE_ADAPTIVE_STATIC_BYTES = 32 << 20
 
 
 class TilemixError(RuntimeError):
@@ -107,6 +112,10 @@ def _load() -> C.CDLL:
     lib.tilemix_route_adaptive.argtypes = [
         vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, i32, i32, i32, vp,
         C.c_size_t, vp, vp, vp, vp]
+    lib.tilemix_route_adaptive_noalloc.restype = i32
+    lib.tilemix_route_adaptive_noalloc.argtypes = [
+        vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, i32, i32, i32, vp,
+        vp, vp, vp]
     lib.tilemix_attn_prefill.restype = i32
     lib.tilemix_attn_prefill.argtypes = [C.POINTER(AttnParams), vp]
     lib.tilemix_status_string.restype = C.c_char_p
@@ -311,6 +320,31 @@ def tilemix_route_adaptive(q, k, cu_seqlens, max_seqlen: int, block_m: int,
         _ptr(route), _ptr(mask), _ptr(status), _stream(stream)),
         "tilemix_route_adaptive")
     return route if mask is None else (route, mask)
+
+
+def tilemix_route_adaptive_noalloc(q, k, cu_seqlens, max_seqlen: int,
+                                   block_m: int, block_n: int, group: int,
+                                   int8_permille: int, *, route, mask=None,
+                                   head_map=None, status=None, stream=None):
+    """tilemix_route_adaptive with the library's static device scratch: the
+    C call allocates nothing (outputs are the caller's: `route` uint8
+    [B, Hkv, Tm, 64] and/or `mask` int64 [B, Hkv, Tm], either may be None).
+    Calls that can overlap on the device share that scratch and must be
+    ordered (one stream, or events)."""
+    torch = _torch()
+    _dev(q, "q", torch.float16)
+    _dev(k, "k", torch.float16)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    _dev(head_map, "head_map", torch.int32)
+    _dev(route, "route", torch.uint8)
+    _dev(mask, "mask", torch.int64)
+    t, hq, d = q.shape
+    _check(lib.tilemix_route_adaptive_noalloc(
+        _ptr(q), _ptr(k), _ptr(cu_seqlens), cu_seqlens.numel() - 1, max_seqlen,
+        t, hq, k.shape[1], d, _ptr(head_map), block_m, block_n, group,
+        int8_permille, _ptr(route), _ptr(mask), _ptr(status), _stream(stream)),
+        "tilemix_route_adaptive_noalloc")
+    return route, mask
 
 
 def tilemix_attn_prefill(q, k, v, cu_seqlens, max_seqlen: int, *, q8=None,

@@ -51,6 +51,10 @@ cudaError_t launch_route_adaptive(const void* q, const void* k,
                                   uint64_t* mask, int32_t* status,
                                   cudaStream_t stream);
 
+// Device address (on the current device) of the file-scope scratch array
+// that tilemix_route_adaptive_noalloc uses; resolved once per device.
+cudaError_t route_adaptive_static_scratch(void** ptr);
+
 // Everything the fused attention kernel reads.  Passed by value as a
 // __grid_constant__ parameter; the tensor maps must stay 64-byte aligned.
 struct AttnParams {

@@ -21,7 +21,10 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "internal.h"
+#include "tilemix.h"
 
 namespace tilemix {
 namespace {
@@ -262,6 +265,32 @@ __global__ void __launch_bounds__(64)
 }
 
 }  // namespace
+
+// Scratch for tilemix_route_adaptive_noalloc: one instance per device
+// context, reserved when this module loads, never allocated per call.  All
+// calls on a device share it, so calls whose work overlaps on the device
+// race on it (the declaration in tilemix.h says how to order them).
+static __device__ __align__(256) unsigned char
+    g_route_scratch[TILEMIX_ROUTE_ADAPTIVE_STATIC_BYTES];
+
+cudaError_t route_adaptive_static_scratch(void** ptr) {
+  constexpr int kCachedDevices = 64;
+  static std::atomic<void*> cached[kCachedDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kCachedDevices) {
+    void* p = cached[dev].load(std::memory_order_acquire);
+    if (p) {
+      *ptr = p;
+      return cudaSuccess;
+    }
+  }
+  e = cudaGetSymbolAddress(ptr, g_route_scratch);
+  if (e == cudaSuccess && dev >= 0 && dev < kCachedDevices)
+    cached[dev].store(*ptr, std::memory_order_release);
+  return e;
+}
 
 size_t route_adaptive_workspace(int batch, int max_seqlen, int hkv, int d,
                                 int block_m) {

@@ -223,42 +223,45 @@ size_t tilemix_route_adaptive_workspace_bytes(int batch, int max_seqlen,
                                            block_m);
 }
 
-tilemix_status tilemix_route_adaptive(
-    const void* q, const void* k, const int32_t* cu_seqlens, int batch,
-    int max_seqlen, int total_tokens, int hq, int hkv, int head_dim,
+namespace {
+
+// Host checks shared by both adaptive-routing entry points.  On TILEMIX_OK,
+// *need is the scratch the two passes use (0 when there is nothing to do).
+tilemix_status route_adaptive_check(
+    const char* where, const void* q, const void* k, const int32_t* cu_seqlens,
+    int batch, int max_seqlen, int total_tokens, int hq, int hkv, int head_dim,
     const int32_t* head_map, int block_m, int block_n, int group,
-    int int8_permille, void* workspace, size_t workspace_bytes,
-    uint8_t* route, uint64_t* mask, int32_t* status, tilemix_stream_t stream) {
+    int int8_permille, const uint8_t* route, const uint64_t* mask,
+    const int32_t* status, size_t* need) {
+  *need = 0;
   if (!q || !k || !cu_seqlens || (!route && !mask))
-    return fail(TILEMIX_ERR_INVALID_ARG, "route_adaptive: null pointer");
+    return fail(TILEMIX_ERR_INVALID_ARG, "%s: null pointer", where);
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(route, 16) ||
-      !aligned(mask, 8) ||
-      !aligned(cu_seqlens, 4) || (head_map && !aligned(head_map, 4)) ||
-      (workspace && !aligned(workspace, 16)) || (status && !aligned(status, 4)))
-    return fail(TILEMIX_ERR_INVALID_ARG, "route_adaptive: misaligned pointer");
+      !aligned(mask, 8) || !aligned(cu_seqlens, 4) ||
+      (head_map && !aligned(head_map, 4)) || (status && !aligned(status, 4)))
+    return fail(TILEMIX_ERR_INVALID_ARG, "%s: misaligned pointer", where);
   if (int8_permille < 0 || int8_permille > 1000)
-    return fail(TILEMIX_ERR_INVALID_ARG,
-                "route_adaptive: int8_permille %d not in [0, 1000]",
-                int8_permille);
+    return fail(TILEMIX_ERR_INVALID_ARG, "%s: int8_permille %d not in [0, 1000]",
+                where, int8_permille);
   if (batch < 0 || max_seqlen < 0 || total_tokens < 0 || hq <= 0 || hkv <= 0 ||
       block_m <= 0 || block_n <= 0 || group <= 0)
-    return fail(TILEMIX_ERR_INVALID_ARG, "route_adaptive: bad size");
+    return fail(TILEMIX_ERR_INVALID_ARG, "%s: bad size", where);
   if (head_dim < 8 || head_dim > 256 || head_dim % 8 != 0)
     return fail(TILEMIX_ERR_UNSUPPORTED,
-                "route_adaptive: head_dim %d not a multiple of 8 in [8, 256]",
+                "%s: head_dim %d not a multiple of 8 in [8, 256]", where,
                 head_dim);
   if (!head_map && hq % hkv != 0)
     return fail(TILEMIX_ERR_INVALID_ARG,
-                "route_adaptive: hq %d not a multiple of hkv %d and no head_map",
-                hq, hkv);
+                "%s: hq %d not a multiple of hkv %d and no head_map", where, hq,
+                hkv);
   if (hkv > 65535 || batch > 65535)
-    return fail(TILEMIX_ERR_UNSUPPORTED, "route_adaptive: hkv or batch > 65535");
+    return fail(TILEMIX_ERR_UNSUPPORTED, "%s: hkv or batch > 65535", where);
   if (batch == 0 || max_seqlen == 0) return ok();
   const long long tn = (static_cast<long long>(max_seqlen) + block_n - 1) / block_n;
   if ((tn + group - 1) / group > 64)
     return fail(TILEMIX_ERR_INVALID_ARG,
-                "route_adaptive: ceil(%lld key tiles / g=%d) > 64 routing bits",
-                tn, group);
+                "%s: ceil(%lld key tiles / g=%d) > 64 routing bits", where, tn,
+                group);
   // |fp16 * 2^24| < 2^40, so a tile's query sums stay below 2^40 * rows and
   // a group's key sums below 2^40 * keys; the device's 24-bit limb products
   // and the int128 statistic stay exact within these bounds.
@@ -268,16 +271,34 @@ tilemix_status tilemix_route_adaptive(
       rows * head_dim >= (1ll << 22) || keys * head_dim >= (1ll << 22) ||
       rows * keys * head_dim >= (1ll << 47))
     return fail(TILEMIX_ERR_UNSUPPORTED,
-                "route_adaptive: tile sizes too large for exact statistics");
+                "%s: tile sizes too large for exact statistics", where);
   const long long tm = (static_cast<long long>(max_seqlen) + block_m - 1) / block_m;
   if (static_cast<long long>(batch) * hkv * tm > 0x7fffffffll)
-    return fail(TILEMIX_ERR_UNSUPPORTED, "route_adaptive: too many routing rows");
-  const size_t need = tilemix::route_adaptive_workspace(batch, max_seqlen, hkv,
-                                                        head_dim, block_m);
-  if (!workspace || workspace_bytes < need)
+    return fail(TILEMIX_ERR_UNSUPPORTED, "%s: too many routing rows", where);
+  *need = tilemix::route_adaptive_workspace(batch, max_seqlen, hkv, head_dim,
+                                            block_m);
+  return ok();
+}
+
+}  // namespace
+
+tilemix_status tilemix_route_adaptive(
+    const void* q, const void* k, const int32_t* cu_seqlens, int batch,
+    int max_seqlen, int total_tokens, int hq, int hkv, int head_dim,
+    const int32_t* head_map, int block_m, int block_n, int group,
+    int int8_permille, void* workspace, size_t workspace_bytes,
+    uint8_t* route, uint64_t* mask, int32_t* status, tilemix_stream_t stream) {
+  size_t need = 0;
+  tilemix_status st = route_adaptive_check(
+      "route_adaptive", q, k, cu_seqlens, batch, max_seqlen, total_tokens, hq,
+      hkv, head_dim, head_map, block_m, block_n, group, int8_permille, route,
+      mask, status, &need);
+  if (st != TILEMIX_OK || need == 0) return st;
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < need)
     return fail(TILEMIX_ERR_INVALID_ARG,
-                "route_adaptive: workspace of %zu bytes, %zu needed",
-                workspace ? workspace_bytes : static_cast<size_t>(0), need);
+                "route_adaptive: workspace of %zu bytes (16-byte aligned) "
+                "needed, %zu given",
+                need, workspace ? workspace_bytes : static_cast<size_t>(0));
   tilemix_status d = check_device();
   if (d != TILEMIX_OK) return d;
   cudaError_t e = tilemix::launch_route_adaptive(
@@ -286,6 +307,40 @@ tilemix_status tilemix_route_adaptive(
       mask, status, stream);
   if (e != cudaSuccess)
     return fail(TILEMIX_ERR_CUDA, "route_adaptive launch: %s",
+                cudaGetErrorString(e));
+  return ok();
+}
+
+tilemix_status tilemix_route_adaptive_noalloc(
+    const void* q, const void* k, const int32_t* cu_seqlens, int batch,
+    int max_seqlen, int total_tokens, int hq, int hkv, int head_dim,
+    const int32_t* head_map, int block_m, int block_n, int group,
+    int int8_permille, uint8_t* route, uint64_t* mask, int32_t* status,
+    tilemix_stream_t stream) {
+  size_t need = 0;
+  tilemix_status st = route_adaptive_check(
+      "route_adaptive_noalloc", q, k, cu_seqlens, batch, max_seqlen,
+      total_tokens, hq, hkv, head_dim, head_map, block_m, block_n, group,
+      int8_permille, route, mask, status, &need);
+  if (st != TILEMIX_OK || need == 0) return st;
+  if (need > TILEMIX_ROUTE_ADAPTIVE_STATIC_BYTES)
+    return fail(TILEMIX_ERR_INVALID_ARG,
+                "route_adaptive_noalloc: %zu bytes of scratch needed, the "
+                "static scratch holds %zu",
+                need, static_cast<size_t>(TILEMIX_ROUTE_ADAPTIVE_STATIC_BYTES));
+  tilemix_status d = check_device();
+  if (d != TILEMIX_OK) return d;
+  void* scratch = nullptr;
+  cudaError_t e = tilemix::route_adaptive_static_scratch(&scratch);
+  if (e != cudaSuccess)
+    return fail(TILEMIX_ERR_CUDA, "route_adaptive_noalloc scratch: %s",
+                cudaGetErrorString(e));
+  e = tilemix::launch_route_adaptive(
+      q, k, cu_seqlens, batch, max_seqlen, total_tokens, hq, hkv, head_dim,
+      head_map, block_m, block_n, group, int8_permille, scratch, route, mask,
+      status, stream);
+  if (e != cudaSuccess)
+    return fail(TILEMIX_ERR_CUDA, "route_adaptive_noalloc launch: %s",
                 cudaGetErrorString(e));
   return ok();
 }
