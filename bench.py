@@ -52,17 +52,25 @@ INT8_OVER_FP16 = 2.0  # nominal dense INT8 / FP16 tensor ratio (4.5 / 2.25 P)
 # this bench's own command, keyed by workload and by a hash of the kernel
 # sources the capture ran; a changed kernel reports null until re-captured.
 NCU_TRAFFIC = {
-    ("llama32_3b_b8_L4096_int8_75", "d4db1ec1b0d1043b"): 466_728_448 + 178_692_864,
+    ("llama32_3b_b8_L4096_int8_75", "89d28c2c46af05c3"): 466_568_192 + 177_329_152,
 }
 KERNEL_SOURCES = ("prefill_blockwise_int8_b200/csrc/attn_prefill.cu",
                   "prefill_blockwise_int8_b200/csrc/ptx.cuh",
                   "prefill_blockwise_int8_b200/csrc/internal.h")
 
 
-def kernel_source_hash():
+# the same for the two adaptive-routing kernels (sums + rank, per call)
+ROUTE_SOURCES = ("prefill_blockwise_int8_b200/csrc/route_adaptive.cu",)
+ROUTE_TRAFFIC = {
+    ("llama32_3b_b8_L4096_int8_75", "3191f6e23b13a14a"):
+        268_517_632 + 8_055_808 + 6_310_400,
+}
+
+
+def kernel_source_hash(sources=KERNEL_SOURCES):
     import hashlib
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in sources:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -70,6 +78,10 @@ def kernel_source_hash():
 
 def measured_traffic(workload_name):
     return NCU_TRAFFIC.get((workload_name, kernel_source_hash()))
+
+
+def measured_route_traffic(workload_name):
+    return ROUTE_TRAFFIC.get((workload_name, kernel_source_hash(ROUTE_SOURCES)))
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -528,6 +540,7 @@ def run_gpu(args):
                       "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                       "frac": round(gbs / float(peaks["hbm_gbs"]), 4),
                       "bytes_per_launch": nbytes,
+                      "traffic": measured_route_traffic(w.name),
                       "kernels": "sums_kernel + rank_kernel"}
 
     cpu = None
