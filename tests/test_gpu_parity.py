@@ -212,6 +212,30 @@ def test_int8_tiles_bitexact_dump(tm, bm, bn, g):
     assert (_mask_past_route_row(dump, lens, bm, bn) != -1).any()
 
 
+@pytest.mark.parametrize("bm,bn,g", [(128, 64, 1), (64, 64, 2)])
+def test_visited_tiles_are_exactly_the_legal_set(tm, bm, bn, g):
+    # every group INT8 and junk bits set in every illegal group: the INT32
+    # dump (filled with -1 first) is written for every legal tile and for
+    # nothing above the diagonal or past a sequence end
+    inp = small([700, 300, 129], bm=bm, bn=bn, g=g, hkv=1, recipe="exact",
+                cov=1.0)
+    w = inp["workload"]
+    junk = W.route_bytes(w, inp["seqlens"], junk_in_illegal=True)
+    got = run_gpu(inp, route=junk, want_dump=True)
+    assert got["status"] == 0
+    _, kw = run_oracle(inp, rows=np.array([0]))
+    dump = oracle.qk_dump(inp["cu_seqlens"], 700, kw["q8"], kw["k8"],
+                          kw["mask"], hq=4, hkv=1, d=128, block_m=bm,
+                          block_n=bn, group=g, fill=-1)
+    lens = inp["seqlens"]
+    ref = _mask_past_route_row(dump, lens, bm, bn)
+    assert np.array_equal(_mask_past_route_row(got["dump"], lens, bm, bn), ref)
+    # nearly every entry of a legal tile holds a dot product (an exact -1 is
+    # possible but rare), so the check above covers the whole legal set
+    legal_pairs = 4 * sum(L * (L + 1) // 2 for L in lens.tolist())
+    assert (ref != -1).sum() >= 0.99 * legal_pairs
+
+
 def test_garbage_bits_in_illegal_groups_change_nothing(tm):
     inp = small([777, 200], bm=128, bn=64, recipe="exact", cov=0.5)
     clean = run_gpu(inp)["out"]
