@@ -11,7 +11,9 @@
 // registers with 16-byte loads, reduces the absmax, and writes the codes
 // with 8-byte stores.  Rows of a block are strided by heads * d in memory,
 // each row contiguous.  The per-element IEEE division is replaced by a
-// multiply with the reciprocal wherever that provably gives the same code.
+// multiply with the reciprocal wherever that provably gives the same code,
+// and the integer code is read off a float's bit pattern (no conversion
+// instruction).
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -91,16 +93,20 @@ __global__ void __launch_bounds__(kQThreads)
     if (idx < nv) {
       const int r = idx / vpr;
       const int c = idx % vpr;
-      const __half* hv = reinterpret_cast<const __half*>(&v[k]);
-      uint32_t packed[2] = {0u, 0u};
+      const uint32_t w4[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+      float f[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int q =
-            amax != 0.0f ? quant_code(__half2float(hv[e]), s, rcp) : 0;
-        packed[e >> 2] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (e & 3));
-      }
+      for (int e = 0; e < 4; ++e) half2_bits_to_float2(w4[e], f[2 * e], f[2 * e + 1]);
+      uint32_t cb[8];
+      quant_codes8(f, s, rcp, cb);
+      // low bytes of four patterns -> one word
+      auto pack4 = [](uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+        return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040),
+                           0x5410);
+      };
       *reinterpret_cast<uint2*>(qbase + r * row_stride + c * 8) =
-          make_uint2(packed[0], packed[1]);
+          make_uint2(pack4(cb[0], cb[1], cb[2], cb[3]),
+                     pack4(cb[4], cb[5], cb[6], cb[7]));
     }
   }
 }
