@@ -77,6 +77,13 @@ enum { TILEMIX_KV_FP16 = 0, TILEMIX_KV_INT8 = 1 };
  * not read (may be NULL).  TILEMIX_KV_FP16 only. */
 #define TILEMIX_FLAG_QUANT_ON_CHIP 2u
 
+/* Test only: the kernel withholds the first V tile of every CTA, so the
+ * consumers' bounded pipeline wait expires (after about 2 s): the call
+ * reports TILEMIX_ERR_TIMEOUT in *status, writes no defined output, and the
+ * context stays usable.  It exercises the timeout path; no fault, trap or
+ * unbounded wait is involved.  Not for production calls. */
+#define TILEMIX_FLAG_TEST_EXPIRE_WAIT 4u
+
 /*
  * Blockwise symmetric INT8 quantisation ("quantize-once").
  * Pages: section 3 Preliminaries (blockwise quantization; INT8 tensor cores

@@ -28,7 +28,7 @@ __all__ = [
     "tilemix_route_adaptive_workspace_bytes", "tilemix_route_adaptive_noalloc",
     "ROUTE_ADAPTIVE_STATIC_BYTES", "tilemix_status_string",
     "tilemix_last_error", "tilemix_version", "KV_FP16", "KV_INT8", "FLAG_FP16_ONLY",
-    "FLAG_QUANT_ON_CHIP", "STATUS",
+    "FLAG_QUANT_ON_CHIP", "FLAG_TEST_EXPIRE_WAIT", "STATUS",
     "LAYOUTS",
 ]
 
@@ -37,6 +37,7 @@ _LIB_PATH = Path(__file__).resolve().parent / "libtilemix.so"
 KV_FP16, KV_INT8 = 0, 1
 FLAG_FP16_ONLY = 1
 FLAG_QUANT_ON_CHIP = 2
+FLAG_TEST_EXPIRE_WAIT = 4  # test only: makes a bounded device wait expire
 STATUS = {0: "TILEMIX_OK", 1: "TILEMIX_ERR_INVALID_ARG",
           2: "TILEMIX_ERR_UNSUPPORTED", 3: "TILEMIX_ERR_CUDA",
           4: "TILEMIX_ERR_TIMEOUT", 5: "TILEMIX_ERR_BAD_SEQLENS",
@@ -354,7 +355,8 @@ def tilemix_attn_prefill(q, k, v, cu_seqlens, max_seqlen: int, *, q8=None,
                          quant_block_q: int = 128, quant_block_k: int = 128,
                          softmax_scale: float = 0.0, head_map=None,
                          fp16_only: bool = False, kv_format: int = KV_FP16,
-                         quant_on_chip: bool = False, out=None, lse=None,
+                         quant_on_chip: bool = False,
+                         test_expire_wait: bool = False, out=None, lse=None,
                          qk_dump=None, status=None, stream=None):
     """Causal tile-routed attention.  q fp16 [T, hq, d]; k, v fp16
     [T, hkv, d] (or k8/v8 int8 + scales with kv_format=KV_INT8).
@@ -385,7 +387,8 @@ def tilemix_attn_prefill(q, k, v, cu_seqlens, max_seqlen: int, *, q8=None,
     p.struct_size = C.sizeof(AttnParams)
     p.kv_format = kv_format
     p.flags = (FLAG_FP16_ONLY if fp16_only else 0) | \
-        (FLAG_QUANT_ON_CHIP if quant_on_chip else 0)
+        (FLAG_QUANT_ON_CHIP if quant_on_chip else 0) | \
+        (FLAG_TEST_EXPIRE_WAIT if test_expire_wait else 0)
     p.q, p.q8, p.q_scale = _ptr(q), _ptr(q8), _ptr(q_scale)
     p.k, p.k8, p.k_scale = _ptr(k), _ptr(k8), _ptr(k_scale)
     p.v, p.v8, p.v_scale = _ptr(v), _ptr(v8), _ptr(v_scale)

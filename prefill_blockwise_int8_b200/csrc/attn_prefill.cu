@@ -542,6 +542,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
           tma_load_3d(sQ8(t), &p.tm_q8, &bars[C::kBarQ], 0, qrow, h);
       }
       int k_issued = 0, v_issued = 0;
+      bool v_withheld = false;
       bool ok = true;
       for (int n = 0; n <= n_end && ok; ++n) {
         const int krow = start + n * kBN;
@@ -579,6 +580,12 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
           ok = false;
           break;
         }
+        // Timeout-path test: V tile 0 is never loaded, so its barrier never
+        // completes and the MMA issuer's bounded wait on it expires.
+        if (n == 0 && p.test_expire_wait) {
+          v_withheld = true;
+          continue;
+        }
         if (KV8) {
           mbar_arrive_expect_tx(&bars[C::kBarV + vs], C::kV8Bytes);
           tma_load_3d(vslot(vs) + C::kV8Off, &p.tm_v8, &bars[C::kBarV + vs], 0,
@@ -599,8 +606,9 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
           mbar_wait(&bars[C::kBarK + n % C::kKStages], (n / C::kKStages) & 1,
                     nullptr);
         for (int n = max(0, v_issued - C::kVStages); n < v_issued; ++n)
-          mbar_wait(&bars[C::kBarV + n % C::kVStages], (n / C::kVStages) & 1,
-                    nullptr);
+          if (!(n == 0 && v_withheld))
+            mbar_wait(&bars[C::kBarV + n % C::kVStages], (n / C::kVStages) & 1,
+                      nullptr);
       }
     }
   } else if (warp == kWarpMma) {

@@ -85,6 +85,7 @@ struct AttnParams {
   int tiles_per_bit; // 64-key blocks per routing bit = g * route_bn / 64
   int quant_block_q, quant_block_k, nbq, nbk;
   int fp16_only;
+  int test_expire_wait;  // withhold the first V tile (timeout-path test)
   float scale_log2;  // softmax scale * log2(e)
 };
 

@@ -357,7 +357,8 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   const bool fp16_only = (a->flags & TILEMIX_FLAG_FP16_ONLY) != 0;
   // With every tile FP16 there is nothing to quantise on chip.
   const bool on_chip = !fp16_only && (a->flags & TILEMIX_FLAG_QUANT_ON_CHIP) != 0;
-  if (a->flags & ~(TILEMIX_FLAG_FP16_ONLY | TILEMIX_FLAG_QUANT_ON_CHIP))
+  if (a->flags & ~(TILEMIX_FLAG_FP16_ONLY | TILEMIX_FLAG_QUANT_ON_CHIP |
+                   TILEMIX_FLAG_TEST_EXPIRE_WAIT))
     return fail(TILEMIX_ERR_INVALID_ARG, "attn: unknown flag bits 0x%x",
                 a->flags);
   if (a->kv_format != TILEMIX_KV_FP16 && a->kv_format != TILEMIX_KV_INT8)
@@ -493,6 +494,7 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   p.nbq = (a->max_seqlen + qbq - 1) / qbq;
   p.nbk = (a->max_seqlen + qbk - 1) / qbk;
   p.fp16_only = fp16_only ? 1 : 0;
+  p.test_expire_wait = (a->flags & TILEMIX_FLAG_TEST_EXPIRE_WAIT) ? 1 : 0;
   const float scale =
       a->softmax_scale > 0.0f ? a->softmax_scale : 1.0f / std::sqrt(float(d));
   p.scale_log2 = scale * 1.4426950408889634f;

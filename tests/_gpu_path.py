@@ -28,7 +28,8 @@ def dev_tensor(a):
 
 
 def run_gpu(inp, *, fp16_only=False, want_lse=False, want_dump=False,
-            head_map=None, stream=None, route=None, on_chip=False):
+            head_map=None, stream=None, route=None, on_chip=False,
+            expire_wait=False):
     """Quantise Q and K, pack the routing words and run attention on the GPU.
     Returns numpy copies of everything the path produced."""
     torch = torch_mod()
@@ -71,7 +72,7 @@ def run_gpu(inp, *, fp16_only=False, want_lse=False, want_dump=False,
         quant_block_q=w.quant_block_q, quant_block_k=w.quant_block_k,
         head_map=hm, fp16_only=fp16_only, lse=lse, qk_dump=dump,
         kv_format=tm.KV_INT8 if kv8 else tm.KV_FP16, status=status,
-        stream=stream)
+        test_expire_wait=expire_wait, stream=stream)
     torch.cuda.synchronize()
     res = dict(status=int(status.item()),
                out=out.float().cpu().numpy().astype(np.float64),

@@ -236,6 +236,25 @@ def test_visited_tiles_are_exactly_the_legal_set(tm, bm, bn, g):
     assert (ref != -1).sum() >= 0.99 * legal_pairs
 
 
+def test_expired_wait_reports_timeout_and_the_context_survives(tm):
+    # the test-only flag withholds every CTA's first V tile: the MMA
+    # issuer's bounded wait expires (about 2 s), the kernel reports
+    # TILEMIX_ERR_TIMEOUT and exits cleanly; later calls work as before
+    inp = small([300, 129], recipe="exact", cov=0.5)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    got = run_gpu(inp, expire_wait=True)
+    t1.record()
+    torch.cuda.synchronize()
+    assert got["status"] == 4            # TILEMIX_ERR_TIMEOUT
+    assert t0.elapsed_time(t1) < 30e3    # bounded: no wait outlives its limit
+    again = run_gpu(inp)
+    assert again["status"] == 0
+    ref, _ = run_oracle(inp)
+    compare(again["out"], ref)
+
+
 def test_garbage_bits_in_illegal_groups_change_nothing(tm):
     inp = small([777, 200], bm=128, bn=64, recipe="exact", cov=0.5)
     clean = run_gpu(inp)["out"]
