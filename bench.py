@@ -12,7 +12,8 @@ words, and the fused attention kernel.  Reported:
               roofline t_roof = (QK_fp16 + PV) / P_fp16 + QK_int8 / P_int8
   e2e         the same metric through the public API with host buffers:
               pinned host -> device copies of Q, K, V and the routing bytes and
-              the device -> host copy of the output inside the timed region
+              the device -> host copy of the output inside the timed region,
+              steps pipelined over copy-in, compute and copy-out streams
   cpu_baseline  the CPU oracle, timed on this host's cores on a bounded
               sample of the same workload (rank 0, one GPU only)
 
