@@ -53,7 +53,7 @@ INT8_OVER_FP16 = 2.0  # nominal dense INT8 / FP16 tensor ratio (4.5 / 2.25 P)
 # this bench's own command, keyed by workload and by a hash of the kernel
 # sources the capture ran; a changed kernel reports null until re-captured.
 NCU_TRAFFIC = {
-    ("llama32_3b_b8_L4096_int8_75", "c82e8670c27741c5"): 466_603_520 + 177_182_208,
+    ("llama32_3b_b8_L4096_int8_75", "5fe750a12f3edf50"): 466_603_520 + 177_182_208,
 }
 KERNEL_SOURCES = ("prefill_blockwise_int8_b200/csrc/attn_prefill.cu",
                   "prefill_blockwise_int8_b200/csrc/ptx.cuh",

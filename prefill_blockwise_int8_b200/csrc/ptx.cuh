@@ -99,7 +99,7 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 // ---------------------------------------------------------------------------
-// TMA (no multicast anywhere in this library)
+// TMA: every copy targets this CTA's own shared memory
 // ---------------------------------------------------------------------------
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
@@ -118,7 +118,7 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m,
       : "memory");
 }
 
-// 3-D tiled bulk store shared -> global (no multicast): the box at
+// 3-D tiled bulk store shared -> global (one destination): the box at
 // coordinates {c0, c1, c2} of the map's tensor from `src`, in this thread's
 // bulk async-group.  c0 * element size must be a multiple of 16 bytes and
 // no coordinate may be negative.
