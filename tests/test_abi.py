@@ -205,3 +205,18 @@ def test_route_adaptive_host_checks():
     assert ra(*args(bn=1 << 15)) == UNSUPPORTED    # limbs could leave int32
     assert ra(*args(hq=512, hkv=2, bm=128)) == UNSUPPORTED   # rows * d >= 2^22
     assert ra(*args(batch=0, max_seqlen=0, ws=None, ws_bytes=0)) == OK
+
+
+def test_every_compute_entry_point_cites_its_passage():
+    # each declaration of a call that launches work is preceded by a comment
+    # naming the passage of the pages it implements (or saying it has none)
+    src = open(HEADER).read()
+    utility = {"tilemix_status_string", "tilemix_last_error", "tilemix_version",
+               "tilemix_route_adaptive_workspace_bytes"}
+    for name in declared_functions():
+        if name in utility:
+            continue
+        decl = re.search(r"\n[a-z_ ]+\*?\s*" + name + r"\s*\(", src)
+        assert decl, name
+        comment = src[:decl.start()].rsplit("*/", 1)[0].rsplit("/*", 1)[1]
+        assert "Pages:" in comment or "No counterpart" in comment, name
