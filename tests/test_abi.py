@@ -220,3 +220,28 @@ def test_every_compute_entry_point_cites_its_passage():
         assert decl, name
         comment = src[:decl.start()].rsplit("*/", 1)[0].rsplit("/*", 1)[1]
         assert "Pages:" in comment or "No counterpart" in comment, name
+
+
+def test_binding_refuses_host_tensors_no_cpu_fallback():
+    torch = pytest.importorskip("torch")
+    x = torch.zeros((4, 2, 64), dtype=torch.float16)
+    k = torch.zeros((4, 1, 64), dtype=torch.float16)
+    cu = torch.tensor([0, 4], dtype=torch.int32)
+    route = torch.zeros((1, 1, 1, 64), dtype=torch.uint8)
+    calls = [
+        lambda: tm.tilemix_quantize_blockwise(x, cu, 4, 128),
+        lambda: tm.tilemix_pack_mask(route, cu, 4, 64, 64, 1),
+        lambda: tm.tilemix_route_template("band", 500, cu, 4, 1, 64, 64, 1),
+        lambda: tm.tilemix_route_adaptive(x, k, cu, 4, 64, 64, 1, 500),
+        lambda: tm.tilemix_attn_prefill(x, k, k, cu, 4, fp16_only=True,
+                                        block_m=64, block_n=64),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            call()
+
+
+def test_missing_library_fails_loudly():
+    stand_in = tm._Missing(OSError("not built"))
+    with pytest.raises(ImportError, match="build"):
+        stand_in.tilemix_attn_prefill
