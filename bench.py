@@ -137,7 +137,10 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def workload_config(w, inp, share):
+def workload_config(w, inp, share, on_chip=False, adaptive=False,
+                    permille=None):
+    """The line's config; both arms (GPU and the CPU oracle) report the same
+    keys for the same workload and options."""
     lens = inp["seqlens"]
     return {
         "workload": w.name,
@@ -154,6 +157,10 @@ def workload_config(w, inp, share):
                                     if w.outliers else ""),
         "parallelism": "replicas",
         "l2": "flushed (256 MiB write) before every timed step",
+        "quantisation": "on chip" if on_chip else "quantise once",
+        "routing": ("adaptive (on device, exact logit-sum statistic, "
+                    f"{permille} permille INT8)" if adaptive
+                    else "given routing bytes"),
     }
 
 
@@ -589,11 +596,9 @@ def run_gpu(args):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp16+int8", "data": "synthetic",
-        "config": dict(workload_config(w, inp, wk["int8_pair_share"]),
-                       quantisation="on chip" if on_chip else "quantise once",
-                       routing=("adaptive (on device, exact logit-sum "
-                                f"statistic, {permille} permille INT8)"
-                                if adaptive else "given routing bytes")),
+        "config": workload_config(w, inp, wk["int8_pair_share"],
+                                  on_chip=on_chip, adaptive=adaptive,
+                                  permille=permille),
         "routing_ms": round(statistics.mean(route_ms), 4),
         "routing_roofline": route_roof,
         "effective_tflops": wk["effective"] / (ms_step * 1e-3) / 1e12 * world,

@@ -231,7 +231,9 @@ tilemix_status tilemix_route_template(
  * head_map) and keys = g * block_n, it needs rows, keys < 2^15, rows * d and
  * keys * d < 2^22, and rows * keys * d < 2^47.  Device side (status word): BAD_SEQLENS for
  * cu_seqlens outside [0, total_tokens] or above max_seqlen, or a head_map
- * entry outside [0, hkv); such a sequence's rows get no FP16 choice.
+ * entry outside [0, hkv).  The rows of such a sequence (with a bad head_map
+ * entry: every row of the call) are not ranked; their route bytes and
+ * routing words are written as 0.
  * Asynchronous on `stream`; allocates nothing.  The workspace query returns
  * 0 for negative or zero sizes.
  */
@@ -247,12 +249,16 @@ tilemix_status tilemix_route_adaptive(
     uint8_t* route, uint64_t* mask, int32_t* status, tilemix_stream_t stream);
 
 /*
- * tilemix_route_adaptive without a caller workspace: the same checks, the
- * same kernels and the same output, with the scratch taken from one static
- * device array of TILEMIX_ROUTE_ADAPTIVE_STATIC_BYTES per device (reserved
- * when the library's module loads on that device; this call allocates
- * nothing, so it may be captured in a CUDA graph).  No counterpart in the
- * TileMix pages: an interface convenience of this library.
+ * tilemix_route_adaptive without a caller workspace, for callers that cannot
+ * allocate device memory themselves: the same checks, the same kernels and
+ * the same output, with the scratch taken from one static device array of
+ * TILEMIX_ROUTE_ADAPTIVE_STATIC_BYTES per device.  The array is reserved
+ * when the library's device code loads on that device, which with CUDA's
+ * lazy module loading happens on the first call of a library kernel there:
+ * make that first call outside any stream capture.  The call itself
+ * allocates nothing; it looks the array's address up in the current context
+ * each time.  No counterpart in the TileMix pages: an interface convenience
+ * of this library.
  *
  * Errors: as tilemix_route_adaptive, and INVALID_ARG when the call would
  * need more than TILEMIX_ROUTE_ADAPTIVE_STATIC_BYTES of scratch

@@ -140,16 +140,29 @@ class _Missing:
                           "with `python -m prefill_blockwise_int8_b200.build`")
 
 
-try:
-    lib = _load()
-except (OSError, AttributeError, ImportError) as _e:
-    lib = _Missing(_e)
+class _Lazy:
+    """The library, mapped into the process on the first attribute access
+    (importing the package, or its host-side helpers such as ``roofline``,
+    maps nothing).  A missing or unusable library raises at that access."""
+
+    def __init__(self):
+        self._lib = None
+
+    def __getattr__(self, name):
+        if self._lib is None:
+            try:
+                self._lib = _load()
+            except (OSError, AttributeError, ImportError) as e:
+                self._lib = _Missing(e)
+        return getattr(self._lib, name)
+
+
+lib = _Lazy()
 
 
 def reload_library():
-    """Load libtilemix.so again (after a build)."""
-    global lib
-    lib = _load()
+    """Load libtilemix.so now (again, after a build); raises if unusable."""
+    lib._lib = _load()
     return lib
 
 

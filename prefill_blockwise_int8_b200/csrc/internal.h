@@ -51,8 +51,8 @@ cudaError_t launch_route_adaptive(const void* q, const void* k,
                                   uint64_t* mask, int32_t* status,
                                   cudaStream_t stream);
 
-// Device address (on the current device) of the file-scope scratch array
-// that tilemix_route_adaptive_noalloc uses; resolved once per device.
+// Device address (in the current context) of the file-scope scratch array
+// that tilemix_route_adaptive_noalloc uses; looked up on every call.
 cudaError_t route_adaptive_static_scratch(void** ptr);
 
 // Everything the fused attention kernel reads.  Passed by value as a

@@ -21,8 +21,6 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
-#include <atomic>
-
 #include "internal.h"
 #include "tilemix.h"
 
@@ -202,7 +200,8 @@ __global__ void __launch_bounds__(kSumThreads)
 // included), and the statistic int128.  Thread j then ranks group j, writes
 // its byte, and warp ballots give the routing word.
 __global__ void __launch_bounds__(64)
-    rank_kernel(const int32_t* __restrict__ cu_seqlens, int max_seqlen,
+    rank_kernel(const int32_t* __restrict__ cu_seqlens,
+                const int32_t* __restrict__ head_map, int hq, int max_seqlen,
                 int total_tokens, int hkv, int tm, int d, int block_m,
                 int block_n, int group, int permille,
                 const int64_t* __restrict__ sq, const int64_t* __restrict__ sk,
@@ -217,8 +216,18 @@ __global__ void __launch_bounds__(64)
   const int b = static_cast<int>(bh / hkv);
   const int start = cu_seqlens[b];
   const int len = cu_seqlens[b + 1] - start;
+  // A head_map entry outside [0, hkv) makes the whole call invalid (the
+  // first pass reported it and left that head out of every sum): every row
+  // is then written as 0, like the rows of an invalid sequence.
+  bool bad_map = false;
+  if (head_map)
+    for (int h = j; h < hq; h += 64) {
+      const int hm = head_map[h];
+      bad_map |= hm < 0 || hm >= hkv;
+    }
+  bad_map = __syncthreads_or(bad_map) != 0;
   int G = 0;  // an invalid sequence was reported by the first pass
-  if (start >= 0 && len >= 0 && len <= max_seqlen &&
+  if (!bad_map && start >= 0 && len >= 0 && len <= max_seqlen &&
       start + len <= total_tokens && static_cast<long long>(m) * block_m < len)
     G = ((min((m + 1) * block_m, len) - 1) / block_n) / group + 1;
   for (int c = j; c < d; c += 64) {
@@ -273,23 +282,13 @@ __global__ void __launch_bounds__(64)
 static __device__ __align__(256) unsigned char
     g_route_scratch[TILEMIX_ROUTE_ADAPTIVE_STATIC_BYTES];
 
+// The array's address in the current context, looked up on every call (a
+// host-side table lookup once the module is loaded): a cached address could
+// outlive its context (a device reset, or another context on the same
+// device) and send the kernels to memory that is no longer theirs.  In host
+// code `g_route_scratch` names a host stand-in, never the device array.
 cudaError_t route_adaptive_static_scratch(void** ptr) {
-  constexpr int kCachedDevices = 64;
-  static std::atomic<void*> cached[kCachedDevices];
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < kCachedDevices) {
-    void* p = cached[dev].load(std::memory_order_acquire);
-    if (p) {
-      *ptr = p;
-      return cudaSuccess;
-    }
-  }
-  e = cudaGetSymbolAddress(ptr, g_route_scratch);
-  if (e == cudaSuccess && dev >= 0 && dev < kCachedDevices)
-    cached[dev].store(*ptr, std::memory_order_release);
-  return e;
+  return cudaGetSymbolAddress(ptr, g_route_scratch);
 }
 
 size_t route_adaptive_workspace(int batch, int max_seqlen, int hkv, int d,
@@ -323,8 +322,8 @@ cudaError_t launch_route_adaptive(const void* q, const void* k,
   if (e != cudaSuccess) return e;
   const long long rows = static_cast<long long>(batch) * hkv * tm;
   rank_kernel<<<static_cast<unsigned>(rows), 64, 0, stream>>>(
-      cu_seqlens, max_seqlen, total_tokens, hkv, tm, d, block_m, block_n, group,
-      permille, sq, sk, route, mask);
+      cu_seqlens, head_map, hq, max_seqlen, total_tokens, hkv, tm, d, block_m,
+      block_n, group, permille, sq, sk, route, mask);
   return cudaGetLastError();
 }
 

@@ -382,10 +382,15 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
     return fail(TILEMIX_ERR_INVALID_ARG,
                 "attn: hq %d not a multiple of hkv %d and no head_map", a->hq,
                 a->hkv);
-  if (a->hq > 65535 || a->batch > 65535 ||
-      (a->max_seqlen + 255) / 256 > 65535)
+  // grid (hq, query-tile groups, batch): a CTA holds 256 query rows, or 128
+  // with 64-row routing words (counted in 64 bits: max_seqlen may be near
+  // INT_MAX)
+  const long long rows_per_cta = a->block_m == 64 ? 128 : 256;
+  const long long cta_rows =
+      (static_cast<long long>(a->max_seqlen) + rows_per_cta - 1) / rows_per_cta;
+  if (a->hq > 65535 || a->batch > 65535 || cta_rows > 65535)
     return fail(TILEMIX_ERR_UNSUPPORTED,
-                "attn: hq, batch or query tiles per sequence above 65535");
+                "attn: hq, batch or query-tile groups per sequence above 65535");
   const int qbq = a->quant_block_q > 0 ? a->quant_block_q : 128;
   const int qbk = a->quant_block_k > 0 ? a->quant_block_k : 128;
   if (qbk % a->block_n != 0)

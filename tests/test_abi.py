@@ -5,6 +5,7 @@ import ctypes as C
 import os
 import re
 import subprocess
+import sys
 import tempfile
 
 import pytest
@@ -245,3 +246,17 @@ def test_missing_library_fails_loudly():
     stand_in = tm._Missing(OSError("not built"))
     with pytest.raises(ImportError, match="build"):
         stand_in.tilemix_attn_prefill
+
+
+def test_import_maps_no_library():
+    # the package and its host-side helpers import without mapping
+    # libtilemix.so; the library loads on the first call into it
+    code = ("import prefill_blockwise_int8_b200 as tm, "
+            "prefill_blockwise_int8_b200.roofline\n"
+            "maps = open('/proc/self/maps').read()\n"
+            "assert 'libtilemix.so' not in maps, 'mapped at import'\n"
+            "tm.lib.tilemix_version\n"
+            "assert 'libtilemix.so' in open('/proc/self/maps').read()\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT,
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr

@@ -335,21 +335,42 @@ def test_int8_kv_cache_needs_its_buffers(tm):
 # full workload sizes, sampled rows
 # ----------------------------------------------------------------------------
 
+def test_full_size_every_row_llama32_3b(tm):
+    # the bench workload (8 x 4096 tokens, 24 / 8 heads, 75% INT8): every
+    # output element against the oracle, and every LSE
+    w = W.LLAMA32_3B_4K
+    inp = W.make(w)
+    got = run_gpu(inp, want_lse=True)
+    assert got["status"] == 0
+    (ref, lse), kw = run_oracle(inp, want_lse=True)
+    assert np.array_equal(got["q8"], kw["q8"])
+    assert np.array_equal(got["k8"], kw["k8"])
+    assert np.array_equal(got["sq"].view(np.uint32), kw["q_scale"].view(np.uint32))
+    assert np.array_equal(got["sk"].view(np.uint32), kw["k_scale"].view(np.uint32))
+    assert np.array_equal(got["mask"], kw["mask"])
+    compare(got["out"], ref)
+    assert np.abs(got["lse"] - lse).max() <= LSE_ABS
+
+
 @pytest.mark.parametrize("wname", [
-    W.LLAMA32_3B_4K.name, W.VARLEN16.name, W.INT8KV_16K.name,
-    W.sweep_32k(75).name, W.sweep_32k(0).name, W.sweep_32k(100).name])
+    W.VARLEN16.name, W.INT8KV_16K.name, W.sweep_32k(0).name,
+    W.sweep_32k(25).name, W.sweep_32k(50).name, W.sweep_32k(75).name,
+    W.sweep_32k(100).name])
 def test_full_size_sampled_rows(tm, wname):
+    # 512 random query rows per sequence (all heads, whole causal rows) plus
+    # the first and last rows of the first, middle and last query tiles
     w = W.WORKLOADS[wname]
     inp = W.make(w)
-    got = run_gpu(inp)
+    got = run_gpu(inp, want_lse=True)
     assert got["status"] == 0
-    rows = sample_rows(inp["seqlens"], inp["cu_seqlens"], per_seq=16,
+    rows = sample_rows(inp["seqlens"], inp["cu_seqlens"], per_seq=512,
                        block=w.block_m)
-    ref, kw = run_oracle(inp, rows=rows)
+    (ref, lse), kw = run_oracle(inp, rows=rows, want_lse=True)
     assert np.array_equal(got["q8"], kw["q8"])
     assert np.array_equal(got["sq"].view(np.uint32), kw["q_scale"].view(np.uint32))
     assert np.array_equal(got["mask"], kw["mask"])
     compare(got["out"], ref, rows=rows)
+    assert np.abs(got["lse"][:, rows] - lse[:, rows]).max() <= LSE_ABS
 
 
 # ----------------------------------------------------------------------------
@@ -373,6 +394,29 @@ def test_route_template_bitexact(tm, layout):
             ref = oracle.route_template(layout, permille, 77, cu, ms, hkv, bm,
                                         bn, g)
             assert np.array_equal(got.cpu().numpy(), ref), (lens, permille)
+
+
+def test_route_template_hash_known_answers(tm):
+    # the device's splitmix64 against the generator's published outputs for
+    # seed 1234567 (tests/golden): with seed = 1234567 - 256 gamma, row 4 of
+    # 64 x 64 tiles hashes exactly the published states 1..5, and row-random
+    # keeps the groups with the largest high halves FP16
+    here = os.path.dirname(__file__)
+    g = json.load(open(os.path.join(here, "golden",
+                                    "splitmix64_known_answers.json")))
+    gamma = int(g["gamma"], 16)
+    seed = (g["seed"] - 256 * gamma) % (1 << 64)
+    hi = [int(v) >> 32 for v in g["outputs"]]
+    by_rank = sorted(range(5), key=lambda j: (-hi[j], j))
+    cu = dev_tensor(np.array([0, 320], np.int32))
+    for permille in (0, 200, 400, 600, 800, 1000):
+        k_int8 = (permille * 5 + 500) // 1000
+        want = np.ones(5, np.uint8)
+        want[by_rank[:5 - k_int8]] = 0
+        got = tm.tilemix_route_template("row_random", permille, cu, 320, 1,
+                                        64, 64, 1, seed=seed)
+        torch.cuda.synchronize()
+        assert np.array_equal(got.cpu().numpy()[0, 0, 4, :5], want), permille
 
 
 def test_route_template_through_attention(tm):
@@ -474,6 +518,24 @@ def test_route_adaptive_bad_seqlens_reported(tm):
     torch.cuda.synchronize()
     assert int(status.item()) == 5     # TILEMIX_ERR_BAD_SEQLENS
     assert not route.cpu().numpy().any()
+
+
+def test_route_adaptive_bad_head_map_reported(tm):
+    # a head_map entry outside [0, hkv): reported, and no row is ranked on
+    # the sums that left that head out (every byte and word written 0)
+    q, k = adaptive_inputs([300, 129], 4, 2, 64, "normal")
+    cu = np.array([0, 300, 429], np.int32)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mask = torch.full((2, 2, 5), -1, dtype=torch.int64, device="cuda")
+    route = torch.full((2, 2, 5, 64), 9, dtype=torch.uint8, device="cuda")
+    tm.tilemix_route_adaptive(dev_tensor(q), dev_tensor(k), dev_tensor(cu),
+                              300, 64, 64, 1, 500,
+                              head_map=dev_tensor(np.array([0, 1, 2, 0], np.int32)),
+                              route=route, mask=mask, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 5     # TILEMIX_ERR_BAD_SEQLENS
+    assert not route.cpu().numpy().any()
+    assert not mask.cpu().numpy().any()
 
 
 def test_route_adaptive_through_attention(tm):

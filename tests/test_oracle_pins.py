@@ -469,6 +469,49 @@ def test_splitmix64_is_a_bijection_on_a_sample():
     assert all(0 <= v < (1 << 64) for v in vals)
 
 
+def _splitmix_golden():
+    with open(os.path.join(GOLDEN, "splitmix64_known_answers.json")) as f:
+        return json.load(f)
+
+
+def test_splitmix64_known_answers():
+    # the published outputs for seed 1234567 (tests/golden, with source)
+    g = _splitmix_golden()
+    gamma = int(g["gamma"], 16)
+    state = g["seed"]
+    for want in g["outputs"]:
+        state = (state + gamma) % (1 << 64)
+        assert oracle.splitmix64(state) == int(want)
+
+
+def test_splitmix64_gamma_is_two_to_64_over_the_golden_ratio():
+    # the increment the templates add per counter step: floor(2^64 / phi)
+    # = floor(2^64 (sqrt 5 - 1) / 2), in exact integer arithmetic
+    import math
+    n = 1 << 64
+    assert (math.isqrt(5 * n * n) - n) // 2 == int(_splitmix_golden()["gamma"], 16)
+
+
+def test_route_template_hash_known_answers():
+    # Row-random ranks a row's groups by the high half of splitmix64 of
+    # seed + (c + 1) * gamma.  With seed = 1234567 - 256 gamma, row m = 4 of
+    # 64 x 64 tiles (c = 256 + j) hashes exactly the published states 1..5,
+    # so the FP16 groups follow from the known outputs alone.
+    g = _splitmix_golden()
+    gamma = int(g["gamma"], 16)
+    seed = (g["seed"] - 256 * gamma) % (1 << 64)
+    hi = [int(v) >> 32 for v in g["outputs"]]
+    by_rank = sorted(range(5), key=lambda j: (-hi[j], j))
+    cu = np.array([0, 320], np.int32)   # row 4 = rows 256..319: 5 groups
+    for permille in (0, 200, 400, 600, 800, 1000):
+        k_int8 = (permille * 5 + 500) // 1000
+        want = np.ones(5, np.uint8)
+        want[by_rank[:5 - k_int8]] = 0
+        got = oracle.route_template("row_random", permille, seed, cu, 320, 1,
+                                    64, 64, 1)[0, 0, 4, :5]
+        assert np.array_equal(got, want), permille
+
+
 # ----------------------------------------------------------------------------
 # adaptive routing: the statistic is the exact sum of raw logits (x 2^48)
 # between a query-tile row and a key group; FP16 goes to the largest
