@@ -239,14 +239,17 @@ __device__ __forceinline__ void exp32(const uint32_t (&sv)[32], float c,
       if (i & 1) xb = fmax3(xb, x.x, x.y);
       else xa = fmax3(xa, x.x, x.y);
     }
-    const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    // P enters P V rounded to fp16; the row sum adds the same rounded
+    // values, so O / l is a weighted mean with exactly the weights P V used
+    const __half2 ph = __floats2half2_rn(ex2_approx(x.x), ex2_approx(x.y));
+    const float2 pr = __half22float2(ph);
     switch (i & 3) {
       case 0: ps0 = __fadd2_rn(ps0, pr); break;
       case 1: ps1 = __fadd2_rn(ps1, pr); break;
       case 2: ps2 = __fadd2_rn(ps2, pr); break;
       default: ps3 = __fadd2_rn(ps3, pr); break;
     }
-    pk[i] = pack_half2(pr.x, pr.y);
+    pk[i] = *reinterpret_cast<const uint32_t*>(&ph);
   }
   if (TRACK) xmax = fmax3(xmax, xa, xb);
 }
