@@ -36,6 +36,7 @@
 #include <math_constants.h>
 #include <stdint.h>
 
+#include "attn_common.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 #include "quant_code.cuh"
@@ -58,9 +59,6 @@ __host__ __device__ constexpr int threads_of(int mode) {
   return mode != kModeGiven ? 640 : 576;
 }
 constexpr int kSmemBudget = 232448;  // max dynamic smem per block on sm_100
-constexpr uint32_t kKindF16 = 1, kKindI8 = 2;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the
-                                           // row max grows by more than 2^8
 
 __host__ __device__ constexpr int align1k(int x) { return (x + 1023) & ~1023; }
 
@@ -147,27 +145,6 @@ struct Cfg {
   static_assert(kNumBars * 8 + 16 <= kBarBytes, "barrier area");
 };
 
-// K-major fp16 operand stored as D/64 column chunks of [rows][128 B] with
-// the 128-byte swizzle; `chunk_bytes` = rows * 128; ks = K-step of 16.
-__device__ __forceinline__ uint64_t desc_k_f16(uint32_t base, int chunk_bytes,
-                                               int ks) {
-  const uint32_t addr = base + (ks >> 2) * chunk_bytes + (ks & 3) * 32;
-  return smem_desc(addr, 16, 1024, kSwizzle128);
-}
-
-// K-major int8 operand (rows x D bytes); ks = K-step of 32 bytes.
-template <int D>
-__device__ __forceinline__ uint64_t desc_k_i8(uint32_t base, int ks) {
-  return smem_desc(base + ks * 32, 16, 8 * D,
-                   D == 128 ? kSwizzle128 : kSwizzle64);
-}
-
-// MN-major fp16 V tile (128 keys x D) stored as D/64 chunks [128][128 B];
-// ks = K-step of 16 keys.  LBO = chunk stride, SBO = 8 keys.
-__device__ __forceinline__ uint64_t desc_v(uint32_t base, int ks) {
-  return smem_desc(base + ks * 16 * 128, kBN * 128, 1024, kSwizzle128);
-}
-
 // Row max of 64 scores held as raw bits (INT32 accumulators when I8, fp32
 // otherwise).  With MASKED, columns j > hl are left out.  The masked /
 // unmasked choice is made once per 64-key half, not per element.
@@ -252,65 +229,6 @@ __device__ __forceinline__ void exp32(const uint32_t (&sv)[32], float c,
     pk[i] = *reinterpret_cast<const uint32_t*>(&ph);
   }
   if (TRACK) xmax = fmax3(xmax, xa, xb);
-}
-
-// Byte offset inside a tile stored with the 128- (m = 7) or 64-byte (m = 3)
-// swizzle: 16-byte unit bits [4:6] XOR row bits [7:9].
-__device__ __forceinline__ uint32_t swz(uint32_t o, uint32_t m) {
-  return o ^ (((o >> 7) & m) << 4);
-}
-
-// Four int8 (one word) -> two fp16 pairs, exactly: bias the bytes to
-// unsigned, place each under the fp16 exponent of 1024 (0x64xx = 1024 +
-// byte), subtract 1024 + 128.
-__device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo,
-                                             uint32_t& hi) {
-  const uint32_t x = w ^ 0x80808080u;
-  const __half2 bias = __float2half2_rn(1152.0f);
-  uint32_t a = __byte_perm(x, 0x64646464u, 0x4140);
-  uint32_t b = __byte_perm(x, 0x64646464u, 0x4342);
-  __half2 ha = __hsub2(*reinterpret_cast<__half2*>(&a), bias);
-  __half2 hb = __hsub2(*reinterpret_cast<__half2*>(&b), bias);
-  lo = *reinterpret_cast<uint32_t*>(&ha);
-  hi = *reinterpret_cast<uint32_t*>(&hb);
-}
-
-// One key row of an INT8 tile (D bytes at row rr of `src`, swizzled with
-// mask sm, 0 = plain rows) -> the fp16 K-major / V layout: D/64 chunks of
-// [128 rows][128 B] with the 128-byte swizzle.  With SCALE, each value is
-// multiplied by s2 (rounded once to fp16).  The whole row is read before
-// any store, so the fp16 row may overlap the INT8 row it came from.
-template <int D, bool SCALE>
-__device__ __forceinline__ void convert_row(const uint8_t* src, uint32_t sm,
-                                            uint8_t* dst, int rr,
-                                            __half2 s2) {
-  uint4 in[D / 16];
-#pragma unroll
-  for (int u = 0; u < D / 16; ++u)
-    in[u] = *reinterpret_cast<const uint4*>(src + swz(rr * D + u * 16, sm));
-#pragma unroll
-  for (int u = 0; u < D / 16; ++u) {
-    const uint32_t w[4] = {in[u].x, in[u].y, in[u].z, in[u].w};
-    uint32_t h[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) i8x4_to_h2x2(w[i], h[2 * i], h[2 * i + 1]);
-    if (SCALE) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        __half2 v = __hmul2(*reinterpret_cast<__half2*>(&h[i]), s2);
-        h[i] = *reinterpret_cast<uint32_t*>(&v);
-      }
-    }
-    // dims 16u .. 16u+15 -> chunk (16u) / 64, 16-byte units 2u, 2u+1 of it
-    const int c = (16 * u) / 64;
-    const int uo = (2 * u) % 8;
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const uint32_t o = c * 128 * 128 + rr * 128 + (uo + e) * 16;
-      *reinterpret_cast<uint4*>(dst + swz(o, 7)) =
-          make_uint4(h[4 * e], h[4 * e + 1], h[4 * e + 2], h[4 * e + 3]);
-    }
-  }
 }
 
 // Largest |x| of row rr of an fp16 tile stored as D/64 chunks of
@@ -699,7 +617,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks)
           mma_f16_ts(tb + C::kOCol, tb + C::p_col(ks >> 2) + (ks & 3) * 8,
-                     desc_v(vb, ks), idesc_pv, (n > 0 || ks > 0) ? 1u : 0u);
+                     desc_v(vb, kBN * 128, ks), idesc_pv, (n > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&bars[C::kBarO + t]);
         return true;
       };
@@ -753,7 +671,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
           uint8_t* kslot_p = kslot(ks);
 #pragma unroll 1
           for (int rr = ct; rr < kBN; rr += 64)
-            convert_row<D, false>(kslot_p + C::kK8Off, k8_swz, kslot_p, rr,
+            convert_row<D, false, kBN * 128>(kslot_p + C::kK8Off, k8_swz, kslot_p, rr,
                                   __float2half2_rn(1.0f));
           fence_proxy_async_smem();
         }
@@ -778,7 +696,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
           int e = 0;
           frexpf(sv, &e);
           const float pow2 = sv > 0.0f ? ldexpf(1.0f, e - 1) : 0.0f;
-          convert_row<D, true>(vslot_p + C::kV8Off, 0u, vslot_p, rr,
+          convert_row<D, true, kBN * 128>(vslot_p + C::kV8Off, 0u, vslot_p, rr,
                                __float2half2_rn(pow2));
         }
         fence_proxy_async_smem();

@@ -65,6 +65,8 @@ struct AttnParams {
   CUtensorMap tm_v;   // fp16 V  [T, hkv, d], box {64, 128, 1}
   CUtensorMap tm_v8;  // int8 V8 [T, hkv, d], box {d, 128, 1}, no swizzle
   CUtensorMap tm_o;   // fp16 O  [T, hq, d], box {64, 128, 1}, 128B swizzle
+  CUtensorMap tm_kh;  // fp16 K  [T, hkv, d], box {64, 64, 1}, 128B swizzle
+  CUtensorMap tm_kh8; // int8 K8 [T, hkv, d], box {d, 64, 1}
   const int32_t* cu_seqlens;
   const int32_t* head_map;
   const uint64_t* mask;
@@ -99,6 +101,11 @@ struct AttnLaunchShape {
 
 cudaError_t launch_attn_prefill(const AttnParams& p, const AttnLaunchShape& s,
                                 cudaStream_t stream);
+
+// The whole-row kernel (128-row routing words, Q8/K8 given or the INT8 KV
+// cache; d in {64, 128}).
+cudaError_t launch_attn_rows(const AttnParams& p, int head_dim, bool kv8,
+                             cudaStream_t stream);
 
 // Dynamic shared memory and TMEM columns a shape needs (host query).
 int attn_smem_bytes(const AttnLaunchShape& s);

@@ -81,6 +81,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------------------
+// register reallocation between warpgroups (every warp of a warpgroup runs
+// the same one); the shares must add up to the block's launch allocation
+// ---------------------------------------------------------------------------
+
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ---------------------------------------------------------------------------
 // fences
 // ---------------------------------------------------------------------------
 
@@ -246,6 +261,29 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
         "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
+}
+
+// 32 consecutive columns from column `off` into r[off .. off + 31] (off a
+// compile-time multiple of 32 after inlining).
+template <int N>
+__device__ __forceinline__ void tmem_ld32_at(uint32_t taddr, uint32_t (&r)[N],
+                                             int off) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[off + 0]), "=r"(r[off + 1]), "=r"(r[off + 2]), "=r"(r[off + 3]),
+        "=r"(r[off + 4]), "=r"(r[off + 5]), "=r"(r[off + 6]), "=r"(r[off + 7]),
+        "=r"(r[off + 8]), "=r"(r[off + 9]), "=r"(r[off + 10]),
+        "=r"(r[off + 11]), "=r"(r[off + 12]), "=r"(r[off + 13]),
+        "=r"(r[off + 14]), "=r"(r[off + 15]), "=r"(r[off + 16]),
+        "=r"(r[off + 17]), "=r"(r[off + 18]), "=r"(r[off + 19]),
+        "=r"(r[off + 20]), "=r"(r[off + 21]), "=r"(r[off + 22]),
+        "=r"(r[off + 23]), "=r"(r[off + 24]), "=r"(r[off + 25]),
+        "=r"(r[off + 26]), "=r"(r[off + 27]), "=r"(r[off + 28]),
+        "=r"(r[off + 29]), "=r"(r[off + 30]), "=r"(r[off + 31])
+      : "r"(taddr + off));
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr,

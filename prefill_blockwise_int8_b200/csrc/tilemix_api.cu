@@ -457,6 +457,8 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   if (maps && !kv8)
     maps = make_map(&p.tm_k, a->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
                     a->hkv, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+           make_map(&p.tm_kh, a->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
+                    a->hkv, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
            make_map(&p.tm_v, a->v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
                     a->hkv, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (maps && !fp16_only && !on_chip)
@@ -466,7 +468,9 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   // chip for FP16 groups) and V8 (converted to fp16 on chip).
   if (maps && (kv8 || (!fp16_only && !on_chip)))
     maps = make_map(&p.tm_k8, a->k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
-                    a->hkv, d, 128, i8sw);
+                    a->hkv, d, 128, i8sw) &&
+           make_map(&p.tm_kh8, a->k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
+                    a->hkv, d, 64, i8sw);
   if (maps && kv8)
     maps = make_map(&p.tm_v8, a->v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
                     a->hkv, d, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -504,8 +508,16 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
       a->softmax_scale > 0.0f ? a->softmax_scale : 1.0f / std::sqrt(float(d));
   p.scale_log2 = scale * 1.4426950408889634f;
 
-  tilemix::AttnLaunchShape shape{d, a->block_m == 64, kv8 ? 1 : (on_chip ? 2 : 0)};
-  cudaError_t e = tilemix::launch_attn_prefill(p, shape, stream);
+  // 128-row routing words without on-chip quantisation run on the
+  // whole-row kernel; 64-row words and on-chip quantisation on the kernel
+  // whose two softmax warpgroups split each tile's keys.
+  cudaError_t e;
+  if (a->block_m == 128 && !on_chip) {
+    e = tilemix::launch_attn_rows(p, d, kv8, stream);
+  } else {
+    tilemix::AttnLaunchShape shape{d, a->block_m == 64, kv8 ? 1 : (on_chip ? 2 : 0)};
+    e = tilemix::launch_attn_prefill(p, shape, stream);
+  }
   if (e != cudaSuccess)
     return fail(TILEMIX_ERR_CUDA, "attn launch: %s", cudaGetErrorString(e));
   return ok();

@@ -568,16 +568,21 @@ ON_CHIP_CASES = {
 
 @pytest.mark.parametrize("name", sorted(ON_CHIP_CASES))
 def test_quant_on_chip_equals_quantise_once(tm, name):
+    # the INT8 tiles made on chip hold exactly the quantise-once integers
+    # (INT32 dumps identical); both modes' outputs and LSE are within the
+    # tolerance of the oracle (the two modes run different kernels, so their
+    # float rounding may differ)
     lens, kw = ON_CHIP_CASES[name]
     inp = small(lens, **kw)
     once = run_gpu(inp, want_lse=True, want_dump=True)
     chip = run_gpu(inp, want_lse=True, want_dump=True, on_chip=True)
     assert once["status"] == 0 and chip["status"] == 0
     assert np.array_equal(chip["dump"], once["dump"])
-    assert np.array_equal(chip["out"], once["out"])
-    assert np.array_equal(chip["lse"], once["lse"])
-    ref, _ = run_oracle(inp)
+    (ref, lse), _ = run_oracle(inp, want_lse=True)
     compare(chip["out"], ref)
+    compare(once["out"], ref)
+    assert np.abs(chip["lse"] - lse).max() <= LSE_ABS
+    assert np.abs(once["lse"] - lse).max() <= LSE_ABS
 
 
 def test_quant_on_chip_full_size_sampled_rows(tm):
