@@ -31,6 +31,7 @@
 // the other tile's P V and next Q K^T execute.
 #include <cuda.h>
 #include <cuda_fp16.h>
+#include <climits>
 #include <math_constants.h>
 #include <stdint.h>
 
@@ -146,38 +147,69 @@ __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   return d;
 }
 
-// Largest of 64 values x[j0 .. j0+63]; with MASKED, columns j > hl count as
-// -inf (hl relative to j0).
-template <bool MASKED>
-__device__ __forceinline__ float max64f(const float (&x)[128], int j0, int hl) {
-  auto g = [&](int j) {
-    return (!MASKED || j <= hl) ? x[j0 + j] : -CUDART_INF_F;
-  };
-  float a[8];
+// Largest score of the 64-key half sv[j0 .. j0+63] held as raw TMEM bits
+// (INT32 accumulators when I8, fp32 otherwise), scaled by c >= 0 into the
+// log2 domain; with MASKED, columns j > hl (relative to j0) are left out and
+// a half with no legal column gives -inf.  Scaling by c >= 0 keeps the
+// order, so only the maximum is converted.
+template <bool I8, bool MASKED>
+__device__ __forceinline__ float half_max(const uint32_t (&sv)[128], int j0,
+                                          int hl, float c) {
+  if (MASKED && hl < 0) return -CUDART_INF_F;
+  if (I8) {
+    auto g = [&](int j) {
+      return (!MASKED || j <= hl) ? static_cast<int>(sv[j0 + j]) : INT_MIN;
+    };
+    int a[8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) a[k] = fmaxf(g(2 * k), g(2 * k + 1));
+    for (int k = 0; k < 8; ++k) a[k] = max(g(2 * k), g(2 * k + 1));
 #pragma unroll
-  for (int j = 16; j < 64; j += 16)
+    for (int j = 16; j < 64; j += 16)
 #pragma unroll
-    for (int k = 0; k < 8; ++k) a[k] = fmax3f(a[k], g(j + 2 * k), g(j + 2 * k + 1));
-  return fmax3f(fmax3f(a[0], a[1], a[2]), fmax3f(a[3], a[4], a[5]),
-                fmaxf(a[6], a[7]));
+      for (int k = 0; k < 8; ++k)
+        a[k] = __vimax3_s32(a[k], g(j + 2 * k), g(j + 2 * k + 1));
+    const int m = __vimax3_s32(__vimax3_s32(a[0], a[1], a[2]),
+                               __vimax3_s32(a[3], a[4], a[5]), max(a[6], a[7]));
+    return __int2float_rn(m) * c;
+  } else {
+    auto g = [&](int j) {
+      return (!MASKED || j <= hl) ? __uint_as_float(sv[j0 + j]) : -CUDART_INF_F;
+    };
+    float a[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = fmaxf(g(2 * k), g(2 * k + 1));
+#pragma unroll
+    for (int j = 16; j < 64; j += 16)
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        a[k] = fmax3f(a[k], g(j + 2 * k), g(j + 2 * k + 1));
+    return fmax3f(fmax3f(a[0], a[1], a[2]), fmax3f(a[3], a[4], a[5]),
+                  fmaxf(a[6], a[7])) * c;
+  }
 }
 
-// P of 32 keys x[j0 .. j0+31]: 2^(x c - m) rounded to fp16, packed in pairs
-// (key 2i in the low half of pk[i]); the same rounded values are added to
-// the partial sums, so O / l is a weighted mean with exactly the weights
-// P V uses.  With MASKED, columns j > hl give 0.
-template <bool MASKED>
-__device__ __forceinline__ void exp32(const float (&x)[128], int j0, float c,
-                                      float m, int hl, uint32_t (&pk)[16],
-                                      float2& sa, float2& sb) {
+// P of a 32-key chunk held as raw TMEM bits in sv: 2^(s c - m) rounded to
+// fp16, packed in pairs (key 2i in the low half of pk[i]); the same rounded
+// values are added to the partial sums, so O / l is a weighted mean with
+// exactly the weights P V uses.  INT32 scores convert exactly (|acc| <=
+// 127^2 d < 2^24) inside the same pass.  With MASKED, columns j > hl give 0.
+template <bool I8, bool MASKED>
+__device__ __forceinline__ void chunk_exp(const uint32_t (&sv)[32], float c,
+                                          float m, int hl, uint32_t (&pk)[16],
+                                          float2& sa, float2& sb) {
   const float2 c2 = make_float2(c, c);
   const float2 nm2 = make_float2(-m, -m);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int j = 2 * i;
-    float2 e = __ffma2_rn(make_float2(x[j0 + j], x[j0 + j + 1]), c2, nm2);
+    float2 v;
+    if (I8) {
+      v = make_float2(__int2float_rn(static_cast<int>(sv[j])),
+                      __int2float_rn(static_cast<int>(sv[j + 1])));
+    } else {
+      v = make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
+    }
+    float2 e = __ffma2_rn(v, c2, nm2);
     if (MASKED) {  // 2^-inf = 0, also when c == 0
       e.x = (j <= hl) ? e.x : -CUDART_INF_F;
       e.y = (j + 1 <= hl) ? e.y : -CUDART_INF_F;
@@ -187,6 +219,75 @@ __device__ __forceinline__ void exp32(const float (&x)[128], int j0, float c,
     if (i & 1) sb = __fadd2_rn(sb, pr);
     else sa = __fadd2_rn(sa, pr);
     pk[i] = *reinterpret_cast<const uint32_t*>(&ph);
+  }
+}
+
+// Masked tiles (the diagonal and the sequence end): the same work with the
+// causal / end mask, kept out of line so the unmasked loop stays small in
+// the instruction cache.  Row max of the 128 scores at s_addr (TMEM), with
+// columns j > hl left out.
+__device__ __noinline__ float masked_row_max(uint32_t s_addr, bool i80,
+                                             bool i81, float c0, float c1,
+                                             int hl) {
+  uint32_t sv[128];
+  tmem_ld32_at(s_addr, sv, 0);
+  tmem_ld32_at(s_addr, sv, 32);
+  tmem_ld32_at(s_addr, sv, 64);
+  tmem_ld32_at(s_addr, sv, 96);
+  tmem_ld_wait();
+  const float m0 = i80 ? half_max<true, true>(sv, 0, hl, c0)
+                       : half_max<false, true>(sv, 0, hl, c0);
+  const float m1 = i81 ? half_max<true, true>(sv, 64, hl - 64, c1)
+                       : half_max<false, true>(sv, 64, hl - 64, c1);
+  return fmaxf(m0, m1);
+}
+
+// P of the 32-key chunk at s_addr with columns j > hl masked, stored as 16
+// fp16 pairs at p_addr; returns the chunk's row sum of the rounded P.
+__device__ __noinline__ float masked_chunk_exp(uint32_t s_addr, uint32_t p_addr,
+                                               bool i8, float c, float m,
+                                               int hl) {
+  uint32_t s32[32], pk[16];
+  tmem_ld32(s_addr, s32);
+  tmem_ld_wait();
+  float2 sa = make_float2(0.f, 0.f), sb = sa;
+  if (i8) chunk_exp<true, true>(s32, c, m, hl, pk, sa, sb);
+  else chunk_exp<false, true>(s32, c, m, hl, pk, sa, sb);
+  tmem_st16(p_addr, pk);
+  const float2 cs = __fadd2_rn(sa, sb);
+  return cs.x + cs.y;
+}
+
+// O *= alpha (per row) for the D columns of O in TMEM at `o_addr`; a rare
+// path (the running max grew by more than 2^8), kept out of the hot loop.
+template <int D>
+__device__ __noinline__ void rescale_o(uint32_t o_addr, float alpha) {
+#pragma unroll 1
+  for (int oc = 0; oc < D; oc += 32) {
+    uint32_t o[32];
+    tmem_ld32(o_addr + oc, o);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+    tmem_st32(o_addr + oc, o);
+  }
+  tmem_st_wait();
+}
+
+// Test output: the raw INT32 scores of this row's 64-key half at `col`
+// (TMEM columns) to dst[0 .. keys_left); warp-collective loads, per-thread
+// stores (`store` false for rows past the sequence).
+__device__ __noinline__ void dump_half(uint32_t s_addr, int32_t* dst,
+                                       int keys_left, bool store) {
+  uint32_t v[32];
+#pragma unroll 1
+  for (int q = 0; q < 2; ++q) {
+    tmem_ld32(s_addr + 32 * q, v);
+    tmem_ld_wait();
+    if (store)
+      for (int j = 0; j < 32; ++j)
+        if (32 * q + j < keys_left) dst[32 * q + j] = static_cast<int32_t>(v[j]);
   }
 }
 
@@ -237,28 +338,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     return r;
   };
   const RowTile rt0 = tile_of(0), rt1 = tile_of(1);
-  auto rt = [&](int t) -> const RowTile& { return t ? rt1 : rt0; };
+  // Per-tile values by selection, never through a reference: a reference
+  // to a local struct would put it in local memory on the hot paths.
+  auto w_of = [&](int t) { return t ? rt1.w : rt0.w; };
+  auto nl_of = [&](int t) { return t ? rt1.nl : rt0.nl; };
+  auto last_of = [&](int t) { return t ? rt1.n_last : rt0.n_last; };
   const int n_end = max(rt0.n_last, rt1.n_last);
   const int tpb = p.tiles_per_bit;  // 64-key blocks per routing bit
   // Path of 64-key half kh of key tile n for query tile t (0: no legal key).
   auto kind_of = [&](int t, int n, int kh) -> uint32_t {
-    const RowTile& r = rt(t);
     const int n64 = 2 * n + kh;
-    if (n64 > r.nl) return 0u;
-    return ((r.w >> (n64 / tpb)) & 1ull) ? kKindI8 : kKindF16;
+    if (n64 > nl_of(t)) return 0u;
+    return ((w_of(t) >> (n64 / tpb)) & 1ull) ? kKindI8 : kKindF16;
   };
   // K halves of key tile n that some query tile needs, per format.  The
   // INT8 cache always brings the whole K8 tile (the fp16 copy is made from
   // it on chip).
-  auto halves_of = [&](int n, uint32_t& h16, uint32_t& h8) {
-    h16 = h8 = 0u;
+  // Returned packed (h16 | h8 << 2), by value.
+  auto halves_of = [&](int n) -> uint32_t {
+    uint32_t h16 = 0u, h8 = 0u;
+#pragma unroll
     for (int t = 0; t < 2; ++t)
+#pragma unroll
       for (int kh = 0; kh < 2; ++kh) {
         const uint32_t k = kind_of(t, n, kh);
         if (k == kKindF16) h16 |= 1u << kh;
         if (k == kKindI8) h8 |= 1u << kh;
       }
     if (KV8) h8 = 3u;
+    return h16 | (h8 << 2);
   };
 
   // ---- shared memory ----
@@ -357,8 +465,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int n = 0; n <= n_end && ok; ++n) {
         const int krow = start + n * kBN;
-        uint32_t h16, h8;
-        halves_of(n, h16, h8);
+        const uint32_t hh = halves_of(n);
+        const uint32_t h16 = hh & 3u, h8 = hh >> 2;
         const KRec rec = ring.plan(h16, h8);
         // Room in the ring and a free record: wait for the oldest tiles'
         // Q K^T to finish reading their blocks.  Live blocks span
@@ -450,16 +558,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(&bars[C::kBarQ], 0, abort_flag);
       tc_fence_after();
       // base descriptors of the resident Q / Q8 tiles (K-step 0)
-      uint64_t dq16[2], dq8[2];
-      for (int t = 0; t < 2; ++t) {
-        dq16[t] = desc_k_f16(smem_u32(sQ(t)), kBM * 128, 0);
-        dq8[t] = desc_k_i8<D>(smem_u32(sQ8(t)), 0);
-      }
+      const uint64_t dq16_0 = desc_k_f16(smem_u32(sQ(0)), kBM * 128, 0);
+      const uint64_t dq16_1 = desc_k_f16(smem_u32(sQ(1)), kBM * 128, 0);
+      const uint64_t dq8_0 = desc_k_i8<D>(smem_u32(sQ8(0)), 0);
+      const uint64_t dq8_1 = desc_k_i8<D>(smem_u32(sQ8(1)), 0);
       const uint32_t kring_u32 = smem_u32(kring);
       // S_t = Q_t K(n)^T, each 64-key half on its path.  A half no row of
       // tile t can see takes the other half's path when that format's block
       // covers it (one N = 128 chain), else it is skipped.
-      auto issue_qk = [&](int t, int n, const KRec& rec) {
+      auto issue_qk = [&](int t, int n, const KRec rec) {
         const uint32_t k0 = kind_of(t, n, 0);
         uint32_t k1 = kind_of(t, n, 1);
         if (k1 == 0u && ((k0 == kKindF16 && rec.h16 == 3u) ||
@@ -476,37 +583,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 (rec.h16 == 3u ? hoff * (kHalf * 128) : 0u);
           const uint64_t db0 = smem_desc(base, 16, 1024, kSwizzle128);
           const uint64_t db1 = smem_desc(base + rows * 128, 16, 1024, kSwizzle128);
-          const uint64_t da0 = dq16[t];
-          const uint64_t da1 = dq16[t] + ((kBM * 128) >> 4);
+          const uint64_t da0 = t ? dq16_1 : dq16_0;
+          const uint64_t da1 = da0 + ((kBM * 128) >> 4);
           const uint32_t d = tb + hoff * kHalf;
           const uint32_t id = halves16 == 3u ? id16_full : id16_half;
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_f16_ss(d, (ks < 4 ? da0 : da1) + k_step(ks),
-                       (ks < 4 ? db0 : db1) + k_step(ks), id, ks > 0 ? 1u : 0u);
+          // compact loops: this code runs once per tile and must stay small
+          // enough to survive in the instruction cache between tiles
+#pragma unroll 1
+          for (int c = 0; c < D / 64; ++c) {
+            uint64_t a = c ? da1 : da0, bb = c ? db1 : db0;
+#pragma unroll 1
+            for (int k = 0; k < 4; ++k, a += 2, bb += 2)
+              mma_f16_ss(d, a, bb, id, (c | k) ? 1u : 0u);
+          }
         }
         if (halves8) {
           const uint32_t hoff = (halves8 == 2u) ? 1u : 0u;
           const uint32_t base = kring_u32 + rec.pos8 +
                                 (rec.h8 == 3u ? hoff * (kHalf * D) : 0u);
           const uint64_t db = desc_k_i8<D>(base, 0);
-          const uint64_t da = dq8[t];
+          const uint64_t da = t ? dq8_1 : dq8_0;
           const uint32_t d = tb + hoff * kHalf;
           const uint32_t id = halves8 == 3u ? id8_full : id8_half;
-#pragma unroll
-          for (int ks = 0; ks < D / 32; ++ks)
-            mma_i8_ss(d, da + 2 * ks, db + 2 * ks, id, ks > 0 ? 1u : 0u);
+          uint64_t a = da, bb = db;
+#pragma unroll 1
+          for (int ks = 0; ks < D / 32; ++ks, a += 2, bb += 2)
+            mma_i8_ss(d, a, bb, id, ks > 0 ? 1u : 0u);
         }
         mma_commit(&bars[C::kBarS + t]);
       };
       // O_t += P_t(n) V(n), P_t(n) in the first 64 columns of S_t.
       auto issue_pv = [&](int t, int n, uint64_t dv) {
         const uint32_t tb = tmem + t * C::kTileCols;
-        const uint32_t acc0 = n > 0 ? 1u : 0u;
-#pragma unroll
-        for (int ks = 0; ks < kBN / 16; ++ks)
-          mma_f16_ts(tb + C::kOCol, tb + ks * 8, dv + ks * (16 * 128 / 16),
-                     idesc_pv, ks > 0 ? 1u : acc0);
+        uint32_t acc = n > 0 ? 1u : 0u;
+        uint32_t pa = tb;
+#pragma unroll 1
+        for (int ks = 0; ks < kBN / 16; ++ks, pa += 8, dv += 16 * 128 / 16) {
+          mma_f16_ts(tb + C::kOCol, pa, dv, idesc_pv, acc);
+          acc = 1u;
+        }
       };
       auto wait_k = [&](int n) -> bool {
         const int s = n % kKRecs;
@@ -523,27 +638,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       KRing<D, C::kKRingBytes> ring;
       KRec rec_next{-1, -1, 0u, 0u};
       {
-        uint32_t h16, h8;
-        halves_of(0, h16, h8);
+        const uint32_t hh = halves_of(0);
+        const uint32_t h16 = hh & 3u, h8 = hh >> 2;
         rec_next = ring.plan(h16, h8);
       }
       if (ok) ok = wait_k(0);
       if (ok) {
         for (int t = 0; t < 2; ++t)
-          if (rt(t).n_last >= 0) issue_qk(t, 0, rec_next);
+          if (last_of(t) >= 0) issue_qk(t, 0, rec_next);
         mma_commit(&bars[C::kBarKEmpty + 0]);
       }
       for (int n = 0; n <= n_end && ok; ++n) {
         KRec rec_n1{-1, -1, 0u, 0u};
         if (n + 1 <= n_end) {
-          uint32_t h16, h8;
-          halves_of(n + 1, h16, h8);
+          const uint32_t hh = halves_of(n + 1);
+          const uint32_t h16 = hh & 3u, h8 = hh >> 2;
           rec_n1 = ring.plan(h16, h8);
         }
         const int vs = n % kVStages;
         bool v_ready = false, k_ready = false;
         for (int t = 0; t < 2 && ok; ++t) {
-          if (n <= rt(t).n_last) {
+          if (n <= last_of(t)) {
             if (!mbar_wait(&bars[C::kBarP + t], n & 1, abort_flag)) {
               ok = false;
               break;
@@ -559,9 +674,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             issue_pv(t, n, desc_v(smem_u32(vslot(vs)), kBN * 128, 0));
-            if (n == rt(t).n_last) mma_commit(&bars[C::kBarO + t]);
+            if (n == last_of(t)) mma_commit(&bars[C::kBarO + t]);
           }
-          if (n + 1 <= rt(t).n_last) {
+          if (n + 1 <= last_of(t)) {
             if (!k_ready) {
               if (!wait_k(n + 1)) {
                 ok = false;
@@ -596,8 +711,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       KRing<D, C::kKRingBytes> ring;
       bool ok = true;
       for (int n = 0; n <= n_end && ok; ++n) {
-        uint32_t h16, h8;
-        halves_of(n, h16, h8);
+        const uint32_t hh = halves_of(n);
+        const uint32_t h16 = hh & 3u, h8 = hh >> 2;
         const KRec rec = ring.plan(h16, h8);
         const int ks = n % kKRecs;
         const bool got_k = mbar_wait(&bars[C::kBarKFull + ks],
@@ -659,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = warp >> 2;
     const int r = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const RowTile& R = rt(t);
+    const RowTile R = t ? rt1 : rt0;  // by value
     bool ok = true;
     if (R.n_last >= 0) {
       const int r_local = row_base + t * kBM + r;
@@ -727,12 +842,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool i80 = kind_of(t, n, 0) == kKindI8;
         const bool i81 = kind_of(t, n, 1) == kKindI8 ||
                          (kind_of(t, n, 1) == 0u && i80);
-        if (p.qk_dump && r_local < len) {
+        if (p.qk_dump) {
           for (int kh = 0; kh < 2; ++kh) {
             const int n64 = 2 * n + kh;
-            if (!(kh ? i81 : i80) || n64 > R.nl) continue;
-            const int rrow = r_local / p.route_bm;
-            const int rr = r_local - rrow * p.route_bm;
+            if (!(kh ? i81 : i80) || n64 > R.nl) continue;  // uniform
+            const int rr_all = min(r_local, len - 1);  // rows past len store nothing
+            const int rrow = rr_all / p.route_bm;
+            const int rr = rr_all - rrow * p.route_bm;
             const int key0 = n64 * kHalf;
             const int nr = key0 / p.route_bn;
             int32_t* dst =
@@ -744,53 +860,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                  rr) *
                     p.route_bn +
                 (key0 - nr * p.route_bn);
-            const int keys_left = len - key0;
-#pragma unroll
-            for (int j = 0; j < kHalf; ++j)
-              if (j < keys_left) dst[j] = static_cast<int32_t>(sv[kh * kHalf + j]);
+            dump_half(lane_addr + kh * kHalf, dst, len - key0, r_local < len);
           }
         }
-        // INT32 scores to fp32 (exact: |acc| <= 127^2 d < 2^24)
-        float x[128];
-#pragma unroll
-        for (int j = 0; j < kHalf; ++j)
-          x[j] = i80 ? __int2float_rn(static_cast<int>(sv[j])) : __uint_as_float(sv[j]);
-#pragma unroll
-        for (int j = kHalf; j < kBN; ++j)
-          x[j] = i81 ? __int2float_rn(static_cast<int>(sv[j])) : __uint_as_float(sv[j]);
         // score scale per half: INT8 sq sk scale log2(e); FP16 scale
         // log2(e) (the INT8 cache's fp16 K is k8, so sk joins)
         const float c0 = i80 ? cq * c_sk0 : (KV8 ? p.scale_log2 * c_sk0 : p.scale_log2);
         const float c1 = i81 ? cq * c_sk1 : (KV8 ? p.scale_log2 * c_sk1 : p.scale_log2);
         const int hl = key_lim - n * kBN;  // legal columns: j <= hl
-        float mx0, mx1;
-        if (hl >= kBN - 1) {
-          mx0 = max64f<false>(x, 0, 0);
-          mx1 = max64f<false>(x, kHalf, 0);
+        // The path of a half is the same for every row of the tile (one
+        // routing word), so these branches are uniform across the warp.
+        // The masked path loads from TMEM itself (warp-collective
+        // tcgen05.ld), so the choice is made per warp: a warp with any
+        // masked row takes the masked path for all its rows (it is exact for
+        // unmasked rows too).
+        float mt;
+        if (__all_sync(0xffffffffu, hl >= kBN - 1)) {
+          const float mx0 = i80 ? half_max<true, false>(sv, 0, 0, c0)
+                                : half_max<false, false>(sv, 0, 0, c0);
+          const float mx1 = i81 ? half_max<true, false>(sv, kHalf, 0, c1)
+                                : half_max<false, false>(sv, kHalf, 0, c1);
+          mt = fmaxf(mx0, mx1);
         } else {
-          mx0 = max64f<true>(x, 0, hl);
-          mx1 = max64f<true>(x, kHalf, hl - kHalf);
+          mt = masked_row_max(lane_addr, i80, i81, c0, c1, hl);
         }
-        // c >= 0, so scaling keeps the order; a fully masked half is -inf
-        const float mt = fmaxf(mx0 == -CUDART_INF_F ? -CUDART_INF_F : mx0 * c0,
-                               mx1 == -CUDART_INF_F ? -CUDART_INF_F : mx1 * c1);
         // Lazy rescaling: keep the old max unless the tile exceeds it by more
         // than 2^threshold, so P <= 2^threshold stays in fp16 range.
         const bool need = mt > m_run + kRescaleThreshold;
         if (n > 0 && __any_sync(0xffffffffu, need)) {
           // S_t(n) is ready, so P V_t(n-1) completed (the MMA thread issues
           // Q K^T_t(n) after it): O_t can be rescaled now.
-          const float alpha = need ? ex2_approx(m_run - mt) : 1.0f;
-#pragma unroll
-          for (int oc = 0; oc < D; oc += 32) {
-            uint32_t o[32];
-            tmem_ld32(lane_addr + C::kOCol + oc, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            tmem_st32(lane_addr + C::kOCol + oc, o);
-          }
+          rescale_o<D>(lane_addr + C::kOCol, need ? ex2_approx(m_run - mt) : 1.0f);
         }
         if (need) {
           l_run *= ex2_approx(m_run - mt);  // 0 while m_run is -inf
@@ -802,22 +902,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (<= 2^9, fp16-safe); the row sum divides f out again.
         const float me0 = KV8 ? m_eff - __log2f(fv0) : m_eff;
         const float me1 = KV8 ? m_eff - __log2f(fv1) : m_eff;
-        float2 sa0 = make_float2(0.f, 0.f), sb0 = sa0, sa1 = sa0, sb1 = sa0;
-#pragma unroll
+        // P, 32 keys at a time (the scores come from TMEM again: one copy of
+        // each chunk's code stays hot in the instruction cache)
+        // the row sum of this tile (with the INT8 cache: P f / f)
+        float lsum = 0.0f;
+        const float rf0 = KV8 ? 1.0f / fv0 : 1.0f, rf1 = KV8 ? 1.0f / fv1 : 1.0f;
+#pragma unroll 1
         for (int q = 0; q < 4; ++q) {
-          uint32_t pk[16];
-          const int j0 = q * 32;
-          const float cc = q < 2 ? c0 : c1;
-          const float mm = q < 2 ? me0 : me1;
-          float2& sa = q < 2 ? sa0 : sa1;
-          float2& sb = q < 2 ? sb0 : sb1;
-          if (hl >= j0 + 31) exp32<false>(x, j0, cc, mm, 0, pk, sa, sb);
-          else exp32<true>(x, j0, cc, mm, hl - j0, pk, sa, sb);
-          tmem_st16(lane_addr + q * 16, pk);
+          const bool h1 = q >= 2;
+          const bool i8 = h1 ? i81 : i80;
+          const float cc = h1 ? c1 : c0;
+          const float mm = h1 ? me1 : me0;
+          const int hq = hl - 32 * q;
+          float cs;
+          if (__all_sync(0xffffffffu, hq >= 31)) {  // warp-uniform, as above
+            uint32_t s32[32], pk[16];
+            tmem_ld32(lane_addr + 32 * q, s32);
+            tmem_ld_wait();
+            float2 sa = make_float2(0.f, 0.f), sb = sa;
+            if (i8) chunk_exp<true, false>(s32, cc, mm, 0, pk, sa, sb);
+            else chunk_exp<false, false>(s32, cc, mm, 0, pk, sa, sb);
+            tmem_st16(lane_addr + 16 * q, pk);
+            const float2 cs2 = __fadd2_rn(sa, sb);
+            cs = cs2.x + cs2.y;
+          } else {
+            cs = masked_chunk_exp(lane_addr + 32 * q, lane_addr + 16 * q, i8, cc,
+                                  mm, hq);
+          }
+          lsum += cs * (h1 ? rf1 : rf0);
         }
-        const float2 s0 = __fadd2_rn(sa0, sb0), s1 = __fadd2_rn(sa1, sb1);
-        l_run += KV8 ? (s0.x + s0.y) / fv0 + (s1.x + s1.y) / fv1
-                     : (s0.x + s0.y) + (s1.x + s1.y);
+        l_run += lsum;
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
