@@ -102,6 +102,9 @@ struct Cfg {
   // exchange [2][2]
   static constexpr int kAuxOff = kRedOff + kRedBytes;
   static constexpr int kAuxBytes = 128;
+  // Q K^T halves of each query tile for the key tile in K slot s (written
+  // by the producer before the slot's loads, read by the MMA issuer)
+  static constexpr int kCodeOff = kAuxOff + 64;
   static constexpr int kSkRing = 8;
   static constexpr int kBarOff = kAuxOff + kAuxBytes;
   static constexpr int kSmem = kBarOff + kBarBytes + 1024;  // + align slack
@@ -357,6 +360,17 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
     if (n64 <= r.nl1) k |= ((r.w1 >> gi) & 1ull) ? kKindI8 : kKindF16;
     return k;
   };
+  // Q K^T of query tile t, key tile n: bits 0-1 the 64-key halves computed
+  // on the FP16 path, bits 2-3 those on the INT8 path (0: no rows there).
+  auto qk_code = [&](int t, int n) -> uint32_t {
+    if (t >= kQT || n > rt(t).n_last) return 0u;
+    const uint32_t k0 = kinds_of(t, n, 0);
+    uint32_t k1 = kinds_of(t, n, 1);
+    if (k1 == 0) k1 = k0;  // keys past every row: any path will do
+    return ((k0 & kKindF16) ? 1u : 0u) | ((k1 & kKindF16) ? 2u : 0u) |
+           ((k0 & kKindI8) ? 4u : 0u) | ((k1 & kKindI8) ? 8u : 0u);
+  };
+  uint32_t* qk_codes = reinterpret_cast<uint32_t*>(smem + C::kCodeOff);
 
   // ---- shared memory carve-up ----
   auto sQ = [&](int t) { return smem + t * C::kQBytes; };
@@ -470,14 +484,16 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
         // K tile n in every format some query tile routes part of it to
         const int ks = n % C::kKStages;
         const int jk = n / C::kKStages;
+        // routing of this key tile, worked out before waiting for its slot
+        const uint32_t code = qk_code(0, n) | (qk_code(1, n) << 4);
+        uint32_t kinds = ((code & 0x33u) ? kKindF16 : 0u) |
+                         ((code & 0xccu) ? kKindI8 : 0u);
         if (jk > 0 &&
             !mbar_wait(&bars[C::kBarKEmpty + ks], (jk - 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
-        uint32_t kinds = 0;
-        for (int t = 0; t < kQT; ++t)
-          kinds |= kinds_of(t, n, 0) | kinds_of(t, n, 1);
+        qk_codes[ks] = code;
         // The INT8 cache only holds K8 (the converters make the fp16 copy);
         // on-chip quantisation makes K8 from K.
         if (KV8) kinds = kKindI8;
@@ -544,22 +560,28 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
       tc_fence_after();
 
       bool q8_ready0 = false, q8_ready1 = false;  // on-chip Q8 seen
+      // Everything the issue path needs is worked out here, so the thread
+      // (which shares its sub-partition with four softmax warps) spends as
+      // few instructions as possible between a barrier and its MMAs:
+      // descriptors are bases plus constant K-step offsets, the routing of
+      // each key tile comes from the producer's code word.
+      const int nl0 = rt0.n_last, nl1 = rt1.n_last;
+      const uint64_t dq16_0 = desc_k_f16(smem_u32(sQ(0)), kBM * 128, 0);
+      const uint64_t dq16_1 = desc_k_f16(smem_u32(sQ(kQT - 1)), kBM * 128, 0);
+      const uint64_t dq8_0 = desc_k_i8<D>(smem_u32(sQ8(0)), 0);
+      const uint64_t dq8_1 = desc_k_i8<D>(smem_u32(sQ8(kQT - 1)), 0);
+      const uint64_t dk16_0 = desc_k_f16(smem_u32(kslot(0)), kBN * 128, 0);
+      const uint64_t dk8_0 = desc_k_i8<D>(smem_u32(kslot(0) + C::kK8Off), 0);
+      const uint64_t dv_0 = desc_v(smem_u32(vslot(0)), kBN * 128, 0);
+      constexpr uint64_t kKSlotStep = C::kKSlotBytes >> 4;  // descriptor units
+      constexpr uint64_t kVSlotStep = C::kVSlotBytes >> 4;
       // S_t(n) = Q_t K(n)^T, each 64-key half on the path(s) it routes to.
       auto issue_qk = [&](int t, int n) -> bool {
-        if (n > rt(t).n_last) return true;
-        const uint32_t k0 = kinds_of(t, n, 0);
-        uint32_t k1 = kinds_of(t, n, 1);
-        if (k1 == 0) k1 = k0;  // keys past every row: any path will do
+        if (n > (t ? nl1 : nl0)) return true;
         const int s = n % C::kKStages;
         if (!mbar_wait(&bars[C::kBarK + s], (n / C::kKStages) & 1, abort_flag))
           return false;
         tc_fence_after();
-        const uint32_t kb = smem_u32(kslot(s));
-        const uint32_t tb = tmem + t * C::kTileCols;
-        const uint32_t halves16 = ((k0 & kKindF16) ? 1u : 0u) |
-                                  ((k1 & kKindF16) ? 2u : 0u);
-        const uint32_t halves8 = ((k0 & kKindI8) ? 1u : 0u) |
-                                 ((k1 & kKindI8) ? 2u : 0u);
         // With converter warps, every key tile waits for them (the fp16 copy
         // of an INT8-cache K tile, or the on-chip K8): the K slot may only
         // free after they passed it, so they never miss a phase of its
@@ -568,6 +590,8 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
             !mbar_wait(&bars[C::kBarKConv + s], (n / C::kKStages) & 1,
                        abort_flag))
           return false;
+        const uint32_t code = (qk_codes[s] >> (4 * t)) & 0xfu;
+        const uint32_t halves16 = code & 3u, halves8 = code >> 2;
         // On-chip quantisation: the converters' Q8 of this tile (once).
         if (QF && halves8) {
           bool& qdone = t ? q8_ready1 : q8_ready0;
@@ -576,35 +600,38 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
           qdone = true;
         }
         if (KV8 || QF) tc_fence_after();
+        const uint32_t tb = tmem + t * C::kTileCols;
+        const uint64_t slot_off = static_cast<uint64_t>(s) * kKSlotStep;
         if (halves16) {
-          const uint32_t q16 = smem_u32(sQ(t));
-          const bool both = halves16 == 3u;
-          const uint32_t hoff = (halves16 == 2u) ? 1u : 0u;  // second half
+          const uint64_t dq = t ? dq16_1 : dq16_0;
+          // one N = 128 chain, or the single 64-key half that needs it
+          const uint32_t hoff = (halves16 == 2u) ? 1u : 0u;
           const uint32_t d = tb + C::kS16 + hoff * kHalf;
-          const uint32_t bk = kb + hoff * (kHalf * 128);  // row 64 of a chunk
+          const uint64_t dk = dk16_0 + slot_off + hoff * (kHalf * 128 / 16);
+          const uint32_t id = halves16 == 3u ? id16_full : id16_half;
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks)
-            mma_f16_ss(d, desc_k_f16(q16, kBM * 128, ks),
-                       desc_k_f16(bk, kBN * 128, ks),
-                       both ? id16_full : id16_half, ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t o = (ks >> 2) * (kBM * 128 / 16) + k_step(ks);
+            const uint64_t ok_ = (ks >> 2) * (kBN * 128 / 16) + k_step(ks);
+            mma_f16_ss(d, dq + o, dk + ok_, id, ks > 0 ? 1u : 0u);
+          }
         }
         if (halves8) {
-          const uint32_t q8 = smem_u32(sQ8(t));
-          const bool both = halves8 == 3u;
+          const uint64_t dq = t ? dq8_1 : dq8_0;
           const uint32_t hoff = (halves8 == 2u) ? 1u : 0u;
           const uint32_t d = tb + C::kS8 + hoff * kHalf;
-          const uint32_t bk = kb + C::kK8Off + hoff * (kHalf * D);
+          const uint64_t dk = dk8_0 + slot_off + hoff * (kHalf * D / 16);
+          const uint32_t id = halves8 == 3u ? id8_full : id8_half;
 #pragma unroll
           for (int ks = 0; ks < D / 32; ++ks)
-            mma_i8_ss(d, desc_k_i8<D>(q8, ks), desc_k_i8<D>(bk, ks),
-                      both ? id8_full : id8_half, ks > 0 ? 1u : 0u);
+            mma_i8_ss(d, dq + ks * 2, dk + ks * 2, id, ks > 0 ? 1u : 0u);
         }
         mma_commit(&bars[C::kBarS + t]);
         return true;
       };
       // O_t += P_t(n) V(n), P_t(n) read from TMEM.
       auto issue_pv = [&](int t, int n) -> bool {
-        if (n > rt(t).n_last) return true;
+        if (n > (t ? nl1 : nl0)) return true;
         const int s = n % C::kVStages;
         if (!mbar_wait(&bars[C::kBarP + t], n & 1, abort_flag)) return false;
         // INT8 cache: the converters' fp16 V (they waited for the TMA)
@@ -612,12 +639,13 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
                        (n / C::kVStages) & 1, abort_flag))
           return false;
         tc_fence_after();
-        const uint32_t vb = smem_u32(vslot(s));
+        const uint64_t dv = dv_0 + static_cast<uint64_t>(s) * kVSlotStep;
         const uint32_t tb = tmem + t * C::kTileCols;
+        const uint32_t acc0 = n > 0 ? 1u : 0u;
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks)
           mma_f16_ts(tb + C::kOCol, tb + C::p_col(ks >> 2) + (ks & 3) * 8,
-                     desc_v(vb, kBN * 128, ks), idesc_pv, (n > 0 || ks > 0) ? 1u : 0u);
+                     dv + ks * (16 * 128 / 16), idesc_pv, ks > 0 ? 1u : acc0);
         mma_commit(&bars[C::kBarO + t]);
         return true;
       };

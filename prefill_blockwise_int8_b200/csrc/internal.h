@@ -102,11 +102,6 @@ struct AttnLaunchShape {
 cudaError_t launch_attn_prefill(const AttnParams& p, const AttnLaunchShape& s,
                                 cudaStream_t stream);
 
-// The whole-row kernel (128-row routing words, Q8/K8 given or the INT8 KV
-// cache; d in {64, 128}).
-cudaError_t launch_attn_rows(const AttnParams& p, int head_dim, bool kv8,
-                             cudaStream_t stream);
-
 // Dynamic shared memory and TMEM columns a shape needs (host query).
 int attn_smem_bytes(const AttnLaunchShape& s);
 

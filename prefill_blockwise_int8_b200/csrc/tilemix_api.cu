@@ -508,16 +508,8 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
       a->softmax_scale > 0.0f ? a->softmax_scale : 1.0f / std::sqrt(float(d));
   p.scale_log2 = scale * 1.4426950408889634f;
 
-  // 128-row routing words without on-chip quantisation run on the
-  // whole-row kernel; 64-row words and on-chip quantisation on the kernel
-  // whose two softmax warpgroups split each tile's keys.
-  cudaError_t e;
-  if (a->block_m == 128 && !on_chip) {
-    e = tilemix::launch_attn_rows(p, d, kv8, stream);
-  } else {
-    tilemix::AttnLaunchShape shape{d, a->block_m == 64, kv8 ? 1 : (on_chip ? 2 : 0)};
-    e = tilemix::launch_attn_prefill(p, shape, stream);
-  }
+  tilemix::AttnLaunchShape shape{d, a->block_m == 64, kv8 ? 1 : (on_chip ? 2 : 0)};
+  const cudaError_t e = tilemix::launch_attn_prefill(p, shape, stream);
   if (e != cudaSuccess)
     return fail(TILEMIX_ERR_CUDA, "attn launch: %s", cudaGetErrorString(e));
   return ok();
