@@ -389,7 +389,7 @@ def run_gpu(args):
     adaptive = args.routing == "adaptive"
     if adaptive and kv8:
         raise SystemExit("--routing adaptive needs fp16 K (not an INT8 KV cache)")
-    launches_per_step = (2 if on_chip else (3 if kv8 else 4)) + \
+    launches_per_step = (2 if on_chip else 3) + \
         (1 if adaptive else 0)
     permille = int(round(w.coverage * 1000))
     ws = None
@@ -405,13 +405,14 @@ def run_gpu(args):
 
     def step(attn_events=None, route_events=None, b=None):
         b = set0 if b is None else b
-        if not on_chip:
+        if not kv8 and not on_chip:  # Q and K in one launch
+            tm.tilemix_quantize_blockwise_qk(
+                b["q"], b["k"], b["cu"], ms, w.quant_block_q, w.quant_block_k,
+                q8=q8, q_scale=sq, k8=b["k8"], k_scale=b["k_scale"],
+                status=status)
+        elif not on_chip:
             tm.tilemix_quantize_blockwise(b["q"], b["cu"], ms, w.quant_block_q,
                                           x8=q8, scale=sq, status=status)
-        if not kv8 and not on_chip:
-            tm.tilemix_quantize_blockwise(b["k"], b["cu"], ms, w.quant_block_k,
-                                          x8=b["k8"], scale=b["k_scale"],
-                                          status=status)
         if route_events:
             route_events[0].record(stream)
         if adaptive:

@@ -84,6 +84,14 @@ enum { TILEMIX_KV_FP16 = 0, TILEMIX_KV_INT8 = 1 };
  * unbounded wait is involved.  Not for production calls. */
 #define TILEMIX_FLAG_TEST_EXPIRE_WAIT 4u
 
+/* Study only (paperlayer summary, appendix G Numerical Analysis: the
+ * deviation of FP16 against FP32 accumulation): the P V product accumulates
+ * O in fp16 in Tensor Memory (kind::f16 MMA with an F16 D format) instead
+ * of fp32; the running max, the row sum and the final O / l stay fp32.
+ * Results are NOT held to the output tolerance of the default mode; the
+ * flag exists to measure how far fp16 accumulation moves the output. */
+#define TILEMIX_FLAG_PV_F16_ACC 8u
+
 /*
  * Blockwise symmetric INT8 quantisation ("quantize-once").
  * Pages: section 3 Preliminaries (blockwise quantization; INT8 tensor cores
@@ -112,6 +120,29 @@ tilemix_status tilemix_quantize_blockwise(
     const void* x, const int32_t* cu_seqlens, int batch, int max_seqlen,
     int total_tokens, int heads, int head_dim, int block, int8_t* x8,
     float* scale, int32_t* status, tilemix_stream_t stream);
+
+/*
+ * Q and K of one attention call quantised in one launch.
+ * Pages: appendix C Quantization Configuration (Q and K quantised blockwise
+ * and symmetrically once per call) and section 3 Preliminaries.
+ * The results are exactly those of tilemix_quantize_blockwise(q, ..., hq,
+ * head_dim, block_q, q8, q_scale) followed by tilemix_quantize_blockwise(k,
+ * ..., hkv, head_dim, block_k, k8, k_scale); one grid covers the blocks of
+ * both tensors.
+ *
+ *   q, k        dev fp16 [T, hq, head_dim] and [T, hkv, head_dim], 16-byte aligned
+ *   q8, k8      dev int8, same shapes, 16-byte aligned
+ *   q_scale     dev fp32 [hq, batch, ceil(max_seqlen / block_q)]
+ *   k_scale     dev fp32 [hkv, batch, ceil(max_seqlen / block_k)]
+ *   block_q, block_k  as `block` above; hq + hkv <= 65535
+ * Errors as for tilemix_quantize_blockwise; nothing is launched when an
+ * argument is rejected.
+ */
+tilemix_status tilemix_quantize_blockwise_qk(
+    const void* q, const void* k, const int32_t* cu_seqlens, int batch,
+    int max_seqlen, int total_tokens, int hq, int hkv, int head_dim,
+    int block_q, int block_k, int8_t* q8, float* q_scale, int8_t* k8,
+    float* k_scale, int32_t* status, tilemix_stream_t stream);
 
 /*
  * Pack per-group routing bytes into 64-bit routing words.

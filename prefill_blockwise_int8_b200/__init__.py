@@ -12,6 +12,8 @@ is missing.
 Entry points (same names as the C ABI):
   tilemix_quantize_blockwise(x, cu_seqlens, max_seqlen, block=128)
       -> (x8, scale)
+  tilemix_quantize_blockwise_qk(q, k, cu_seqlens, max_seqlen) (one launch)
+      -> (q8, q_scale, k8, k_scale)
   tilemix_pack_mask(route, cu_seqlens, max_seqlen, block_m, block_n, group)
       -> mask
   tilemix_attn_prefill(q, k, v, cu_seqlens, max_seqlen, ...) -> out
@@ -23,12 +25,13 @@ from pathlib import Path
 
 __all__ = [
     "TilemixError", "lib", "library_path", "EXPORTED_SYMBOLS",
-    "tilemix_quantize_blockwise", "tilemix_pack_mask", "tilemix_attn_prefill",
+    "tilemix_quantize_blockwise", "tilemix_quantize_blockwise_qk",
+    "tilemix_pack_mask", "tilemix_attn_prefill",
     "tilemix_route_template", "tilemix_route_adaptive",
     "tilemix_route_adaptive_workspace_bytes", "tilemix_route_adaptive_noalloc",
     "ROUTE_ADAPTIVE_STATIC_BYTES", "tilemix_status_string",
     "tilemix_last_error", "tilemix_version", "KV_FP16", "KV_INT8", "FLAG_FP16_ONLY",
-    "FLAG_QUANT_ON_CHIP", "FLAG_TEST_EXPIRE_WAIT", "STATUS",
+    "FLAG_QUANT_ON_CHIP", "FLAG_TEST_EXPIRE_WAIT", "FLAG_PV_F16_ACC", "STATUS",
     "LAYOUTS",
 ]
 
@@ -38,6 +41,7 @@ KV_FP16, KV_INT8 = 0, 1
 FLAG_FP16_ONLY = 1
 FLAG_QUANT_ON_CHIP = 2
 FLAG_TEST_EXPIRE_WAIT = 4  # test only: makes a bounded device wait expire
+FLAG_PV_F16_ACC = 8  # study only: O accumulated in fp16 (no tolerance)
 STATUS = {0: "TILEMIX_OK", 1: "TILEMIX_ERR_INVALID_ARG",
           2: "TILEMIX_ERR_UNSUPPORTED", 3: "TILEMIX_ERR_CUDA",
           4: "TILEMIX_ERR_TIMEOUT", 5: "TILEMIX_ERR_BAD_SEQLENS",
@@ -49,7 +53,8 @@ LAYOUTS = {"all_fp16": 0, "all_int8": 1, "band": 2, "global": 3,
 
 # Every function include/tilemix.h declares.
 EXPORTED_SYMBOLS = (
-    "tilemix_quantize_blockwise", "tilemix_pack_mask", "tilemix_attn_prefill",
+    "tilemix_quantize_blockwise", "tilemix_quantize_blockwise_qk",
+    "tilemix_pack_mask", "tilemix_attn_prefill",
     "tilemix_route_template", "tilemix_route_adaptive_workspace_bytes",
     "tilemix_route_adaptive", "tilemix_route_adaptive_noalloc",
     "tilemix_status_string", "tilemix_last_error", "tilemix_version",
@@ -101,6 +106,10 @@ def _load() -> C.CDLL:
     lib.tilemix_quantize_blockwise.restype = i32
     lib.tilemix_quantize_blockwise.argtypes = [
         vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]
+    lib.tilemix_quantize_blockwise_qk.restype = i32
+    lib.tilemix_quantize_blockwise_qk.argtypes = [
+        vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp,
+        vp, vp]
     lib.tilemix_pack_mask.restype = i32
     lib.tilemix_pack_mask.argtypes = [
         vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
@@ -242,6 +251,42 @@ def tilemix_quantize_blockwise(x, cu_seqlens, max_seqlen: int, block: int = 128,
     return x8, scale
 
 
+def tilemix_quantize_blockwise_qk(q, k, cu_seqlens, max_seqlen: int,
+                                  block_q: int = 128, block_k: int = 128, *,
+                                  q8=None, q_scale=None, k8=None, k_scale=None,
+                                  status=None, stream=None):
+    """Q and K quantised in one launch: returns (q8, q_scale, k8, k_scale),
+    equal to two tilemix_quantize_blockwise calls."""
+    torch = _torch()
+    _dev(q, "q", torch.float16)
+    _dev(k, "k", torch.float16)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    t, hq, d = q.shape
+    tk, hkv, dk = k.shape
+    if (tk, dk) != (t, d):
+        raise ValueError("q and k must share tokens and head_dim")
+    batch = cu_seqlens.numel() - 1
+    if q8 is None:
+        q8 = torch.empty((t, hq, d), dtype=torch.int8, device=q.device)
+    if k8 is None:
+        k8 = torch.empty((t, hkv, d), dtype=torch.int8, device=q.device)
+    if q_scale is None:
+        q_scale = torch.empty((hq, batch, -(-max_seqlen // block_q)),
+                              dtype=torch.float32, device=q.device)
+    if k_scale is None:
+        k_scale = torch.empty((hkv, batch, -(-max_seqlen // block_k)),
+                              dtype=torch.float32, device=q.device)
+    for tns, nm, dt in ((q8, "q8", torch.int8), (k8, "k8", torch.int8),
+                        (q_scale, "q_scale", torch.float32),
+                        (k_scale, "k_scale", torch.float32)):
+        _dev(tns, nm, dt)
+    _check(lib.tilemix_quantize_blockwise_qk(
+        _ptr(q), _ptr(k), _ptr(cu_seqlens), batch, max_seqlen, t, hq, hkv, d,
+        block_q, block_k, _ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale),
+        _ptr(status), _stream(stream)), "tilemix_quantize_blockwise_qk")
+    return q8, q_scale, k8, k_scale
+
+
 def tilemix_pack_mask(route, cu_seqlens, max_seqlen: int, block_m: int,
                       block_n: int, group: int, *, mask=None, status=None,
                       stream=None):
@@ -369,7 +414,8 @@ def tilemix_attn_prefill(q, k, v, cu_seqlens, max_seqlen: int, *, q8=None,
                          softmax_scale: float = 0.0, head_map=None,
                          fp16_only: bool = False, kv_format: int = KV_FP16,
                          quant_on_chip: bool = False,
-                         test_expire_wait: bool = False, out=None, lse=None,
+                         test_expire_wait: bool = False,
+                         pv_f16_acc: bool = False, out=None, lse=None,
                          qk_dump=None, status=None, stream=None):
     """Causal tile-routed attention.  q fp16 [T, hq, d]; k, v fp16
     [T, hkv, d] (or k8/v8 int8 + scales with kv_format=KV_INT8).
@@ -401,7 +447,8 @@ def tilemix_attn_prefill(q, k, v, cu_seqlens, max_seqlen: int, *, q8=None,
     p.kv_format = kv_format
     p.flags = (FLAG_FP16_ONLY if fp16_only else 0) | \
         (FLAG_QUANT_ON_CHIP if quant_on_chip else 0) | \
-        (FLAG_TEST_EXPIRE_WAIT if test_expire_wait else 0)
+        (FLAG_TEST_EXPIRE_WAIT if test_expire_wait else 0) | \
+        (FLAG_PV_F16_ACC if pv_f16_acc else 0)
     p.q, p.q8, p.q_scale = _ptr(q), _ptr(q8), _ptr(q_scale)
     p.k, p.k8, p.k_scale = _ptr(k), _ptr(k8), _ptr(k_scale)
     p.v, p.v8, p.v_scale = _ptr(v), _ptr(v8), _ptr(v_scale)

@@ -65,6 +65,7 @@ __host__ __device__ constexpr int align1k(int x) { return (x + 1023) & ~1023; }
 template <int D, bool DUAL, int MODE>
 struct Cfg {
   static constexpr bool KV8 = MODE == kModeKV8;
+  static constexpr bool QF = MODE == kModeOnChip;
   // DUAL (64-row routing words): a 128-row query tile may need both paths
   // for the same keys, so S has an fp16 and an int8 region and the CTA
   // holds one query tile.
@@ -82,7 +83,12 @@ struct Cfg {
   static constexpr int kQ8Off = kQT * kQBytes;
   static constexpr int kRing0 = align1k(kQ8Off + kQT * kQ8Bytes);
   static constexpr int kK8Off = align1k(kK16Bytes);
-  static constexpr int kKSlotBytes = align1k(kK8Off + kK8Bytes);
+  // On-chip quantisation keeps its K8 tiles in a ring of their own, which
+  // the converter warps fill from K in global memory ahead of the MMAs; its
+  // K slots then hold fp16 K only.
+  static constexpr int kKSlotBytes =
+      QF ? align1k(kK16Bytes) : align1k(kK8Off + kK8Bytes);
+  static constexpr int kK8Ring = QF ? 2 : 0;
   // (d = 64 stages V8 past the fp16 tile: there rows would overlap)
   static constexpr int kVSlotBytes =
       align1k(KV8 && D != 128 ? kVBytes + kBN * D : kVBytes);
@@ -91,12 +97,15 @@ struct Cfg {
   static constexpr int kAvail =
       kSmemBudget - 1024 - kBarBytes - kRedBytes - 128 - kRing0;
   // Two V slots (P V of every query tile must finish before a V slot
-  // frees), then as many K slots as fit (at most 3).
-  static constexpr int kVStages = 2;
-  static constexpr int kKFit = (kAvail - kVStages * kVSlotBytes) / kKSlotBytes;
+  // frees; one beside the on-chip K8 ring, whose V load has a whole softmax
+  // pass to land), then as many K slots as fit (at most 3).
+  static constexpr int kVStages = QF ? 1 : 2;
+  static constexpr int kKFit =
+      (kAvail - kVStages * kVSlotBytes - kK8Ring * kK8Bytes) / kKSlotBytes;
   static constexpr int kKStages = kKFit > 3 ? 3 : kKFit;
   static_assert(kKStages >= 1, "shared memory too small");
-  static constexpr int kVRing0 = kRing0 + kKStages * kKSlotBytes;
+  static constexpr int kK8Ring0 = kRing0 + kKStages * kKSlotBytes;
+  static constexpr int kVRing0 = kK8Ring0 + kK8Ring * kK8Bytes;
   static constexpr int kRedOff = kVRing0 + kVStages * kVSlotBytes;
   // on-chip quantisation: Q scales [2], K-scale ring [8], converter max
   // exchange [2][2]
@@ -143,7 +152,9 @@ struct Cfg {
   static constexpr int kBarQConv = kBarVConv + kVStages;  // [tile]
   static constexpr int kBarSK = kBarQConv + 2;            // [ring slot]
   static constexpr int kBarCvX = kBarSK + kSkRing;
-  static constexpr int kBarDrain = kBarCvX + 1;
+  static constexpr int kBarK8Full = kBarCvX + 1;       // [K8 ring slot]
+  static constexpr int kBarK8Empty = kBarK8Full + 2;   // [K8 ring slot]
+  static constexpr int kBarDrain = kBarK8Empty + 2;
   static constexpr int kNumBars = kBarDrain + 1;
   static_assert(kNumBars * 8 + 16 <= kBarBytes, "barrier area");
 };
@@ -250,30 +261,73 @@ __device__ __forceinline__ float row_absmax_f16(const uint8_t* tile, int rr) {
   return fmaxf(__low2float(m), __high2float(m));
 }
 
+// 16 fp16 values (two 16-byte words) -> their 16 codes as one 16-byte word
+// (code of value i in byte i), with the quantiser's exact definition.
+__device__ __forceinline__ uint4 codes16(uint4 a, uint4 b, float s, float r) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t out[4];
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    float f[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      half2_bits_to_float2(w[4 * hh + e], f[2 * e], f[2 * e + 1]);
+    uint32_t cb[8];
+    quant_codes8(f, s, r, cb);
+    out[2 * hh] = pack_low_bytes4(cb[0], cb[1], cb[2], cb[3]);
+    out[2 * hh + 1] = pack_low_bytes4(cb[4], cb[5], cb[6], cb[7]);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
 // Codes of row rr of that fp16 tile into an INT8 tile of D-byte rows with
-// the swizzle of mask sm (the layout the INT8 MMA reads), scale s, 1/s = r;
-// zero: the block is all zeros (codes 0).
+// the swizzle of mask sm (the layout the INT8 MMA reads), scale s, 1/s = r
+// (a zero block has s = r = 0: codes 0).
 template <int D>
 __device__ __forceinline__ void quant_row(const uint8_t* tile16,
                                           uint8_t* tile8, uint32_t sm, int rr,
-                                          float s, float r, bool zero) {
+                                          float s, float r) {
 #pragma unroll
   for (int v = 0; v < D / 16; ++v) {
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    uint4 x[2];
 #pragma unroll
     for (int hu = 0; hu < 2; ++hu) {
       const int u = 2 * v + hu;
       const uint32_t o = (u / 8) * 128 * 128 + rr * 128 + (u % 8) * 16;
-      const uint4 x = *reinterpret_cast<const uint4*>(tile16 + swz(o, 7));
-      const __half* h = reinterpret_cast<const __half*>(&x);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int q = zero ? 0 : quant_code(__half2float(h[e]), s, r);
-        w[2 * hu + e / 4] |= (static_cast<uint32_t>(q) & 0xffu) << (8 * (e % 4));
-      }
+      x[hu] = *reinterpret_cast<const uint4*>(tile16 + swz(o, 7));
     }
     *reinterpret_cast<uint4*>(tile8 + swz(rr * D + v * 16, sm)) =
-        make_uint4(w[0], w[1], w[2], w[3]);
+        codes16(x[0], x[1], s, r);
+  }
+}
+
+// Largest |x| of one contiguous fp16 row of D values in global memory.
+template <int D>
+__device__ __forceinline__ float row_absmax_global(const __half* row) {
+  __half2 m = __float2half2_rn(0.0f);
+#pragma unroll
+  for (int u = 0; u < D / 8; ++u) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(row) + u);
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) m = __hmax2(m, __habs2(h[e]));
+  }
+  return fmaxf(__low2float(m), __high2float(m));
+}
+
+// Codes of one contiguous fp16 row in global memory (nullptr: a row past
+// the sequence, codes 0) into row rr of an INT8 tile laid out as above.
+template <int D>
+__device__ __forceinline__ void quant_row_global(const __half* row,
+                                                 uint8_t* tile8, uint32_t sm,
+                                                 int rr, float s, float r) {
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int v = 0; v < D / 16; ++v) {
+    const uint4 a = row ? __ldg(reinterpret_cast<const uint4*>(row) + 2 * v) : zero;
+    const uint4 b = row ? __ldg(reinterpret_cast<const uint4*>(row) + 2 * v + 1) : zero;
+    *reinterpret_cast<uint4*>(tile8 + swz(rr * D + v * 16, sm)) =
+        codes16(a, b, s, r);
   }
 }
 
@@ -409,6 +463,10 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
       for (int i = 0; i < 2; ++i) mbar_init(&bars[C::kBarQConv + i], 2);
       for (int i = 0; i < C::kSkRing; ++i) mbar_init(&bars[C::kBarSK + i], 2);
       mbar_init(&bars[C::kBarCvX], 2);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&bars[C::kBarK8Full + i], 2);   // the two converter warps
+        mbar_init(&bars[C::kBarK8Empty + i], 1);  // MMA commit
+      }
     }
     mbar_init(&bars[C::kBarDrain], 1);
     *abort_flag = 0;
@@ -497,7 +555,7 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
         // The INT8 cache only holds K8 (the converters make the fp16 copy);
         // on-chip quantisation makes K8 from K.
         if (KV8) kinds = kKindI8;
-        if (QF) kinds = kKindF16;
+        if (QF) kinds &= kKindF16;  // K8 comes from the converters' ring
         mbar_arrive_expect_tx(&bars[C::kBarK + ks],
                               ((kinds & kKindF16) ? C::kK16Bytes : 0) +
                                   ((kinds & kKindI8) ? C::kK8Bytes : 0));
@@ -555,7 +613,9 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
       constexpr uint32_t id16_half = instr_desc(1, 0, 0, 0, 0, kHalf, kBM);
       constexpr uint32_t id8_full = instr_desc(2, 1, 1, 0, 0, kBN, kBM);
       constexpr uint32_t id8_half = instr_desc(2, 1, 1, 0, 0, kHalf, kBM);
-      constexpr uint32_t idesc_pv = instr_desc(1, 0, 0, 0, 1, D, kBM);
+      // O in fp32, or (study flag) in fp16: one value in the low half of
+      // each TMEM column either way
+      const uint32_t idesc_pv = instr_desc(p.pv_f16_acc ? 0 : 1, 0, 0, 0, 1, D, kBM);
       bool ok = mbar_wait(&bars[C::kBarQ], 0, abort_flag);
       tc_fence_after();
 
@@ -571,7 +631,8 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
       const uint64_t dq8_0 = desc_k_i8<D>(smem_u32(sQ8(0)), 0);
       const uint64_t dq8_1 = desc_k_i8<D>(smem_u32(sQ8(kQT - 1)), 0);
       const uint64_t dk16_0 = desc_k_f16(smem_u32(kslot(0)), kBN * 128, 0);
-      const uint64_t dk8_0 = desc_k_i8<D>(smem_u32(kslot(0) + C::kK8Off), 0);
+      const uint64_t dk8_0 =
+          desc_k_i8<D>(smem_u32(QF ? smem + C::kK8Ring0 : kslot(0) + C::kK8Off), 0);
       const uint64_t dv_0 = desc_v(smem_u32(vslot(0)), kBN * 128, 0);
       constexpr uint64_t kKSlotStep = C::kKSlotBytes >> 4;  // descriptor units
       constexpr uint64_t kVSlotStep = C::kVSlotBytes >> 4;
@@ -586,18 +647,22 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
         // of an INT8-cache K tile, or the on-chip K8): the K slot may only
         // free after they passed it, so they never miss a phase of its
         // full barrier.
-        if ((KV8 || QF) &&
+        if (KV8 &&
             !mbar_wait(&bars[C::kBarKConv + s], (n / C::kKStages) & 1,
                        abort_flag))
           return false;
         const uint32_t code = (qk_codes[s] >> (4 * t)) & 0xfu;
         const uint32_t halves16 = code & 3u, halves8 = code >> 2;
-        // On-chip quantisation: the converters' Q8 of this tile (once).
+        // On-chip quantisation: the converters' Q8 of this tile (once) and
+        // the K8 of this key tile in ring slot n % 2.
         if (QF && halves8) {
           bool& qdone = t ? q8_ready1 : q8_ready0;
           if (!qdone && !mbar_wait(&bars[C::kBarQConv + t], 0, abort_flag))
             return false;
           qdone = true;
+          if (!mbar_wait(&bars[C::kBarK8Full + (n & 1)], (n >> 1) & 1,
+                         abort_flag))
+            return false;
         }
         if (KV8 || QF) tc_fence_after();
         const uint32_t tb = tmem + t * C::kTileCols;
@@ -620,7 +685,9 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
           const uint64_t dq = t ? dq8_1 : dq8_0;
           const uint32_t hoff = (halves8 == 2u) ? 1u : 0u;
           const uint32_t d = tb + C::kS8 + hoff * kHalf;
-          const uint64_t dk = dk8_0 + slot_off + hoff * (kHalf * D / 16);
+          const uint64_t ring_off =
+              QF ? static_cast<uint64_t>(n & 1) * (C::kK8Bytes / 16) : slot_off;
+          const uint64_t dk = dk8_0 + ring_off + hoff * (kHalf * D / 16);
           const uint32_t id = halves8 == 3u ? id8_full : id8_half;
 #pragma unroll
           for (int ks = 0; ks < D / 32; ++ks)
@@ -654,7 +721,10 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
       // P V that reads P of tile n.  A K slot frees when every query tile's
       // Q K^T of it completed, a V slot when every P V did.
       for (int t = 0; t < kQT && ok; ++t) ok = issue_qk(t, 0);
-      if (ok) mma_commit(&bars[C::kBarKEmpty + 0]);
+      if (ok) {
+        mma_commit(&bars[C::kBarKEmpty + 0]);
+        if (QF) mma_commit(&bars[C::kBarK8Empty + 0]);
+      }
       for (int n = 0; n <= n_end && ok; ++n) {
         for (int t = 0; t < kQT && ok; ++t) {
           ok = issue_pv(t, n);
@@ -662,8 +732,10 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
         }
         if (ok) {
           mma_commit(&bars[C::kBarVEmpty + n % C::kVStages]);
-          if (n + 1 <= n_end)
+          if (n + 1 <= n_end) {
             mma_commit(&bars[C::kBarKEmpty + (n + 1) % C::kKStages]);
+            if (QF) mma_commit(&bars[C::kBarK8Empty + ((n + 1) & 1)]);
+          }
         }
       }
       if (!ok) fail();
@@ -735,11 +807,14 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
     }
     if (QF) {
       // =================== on-chip quantisation (2 warps) ===================
-      // Q8 of each query tile once, then K8 of each key tile that some row
-      // routes to INT8, with the quantiser's definition over the block's
-      // rows inside the sequence (a 128-row tile is one 128-token block).
-      // Each thread quantises whole rows (ct and ct + 64); the block max
-      // combines the two warps through shared memory.
+      // Q8 of each query tile once (from Q in shared memory), then K8 of
+      // each key tile that some row routes to INT8, with the quantiser's
+      // definition over the block's rows inside the sequence (a 128-row tile
+      // is one 128-token block).  K rows are read from global memory (L2),
+      // not from the K slot, into a two-slot K8 ring, so the converters run
+      // up to two key tiles ahead of the MMAs instead of waiting for each
+      // fp16 K tile to land.  Each thread quantises whole rows (ct and
+      // ct + 64); the block max combines the two warps through shared memory.
       const int cw = warp - kWarpConv;
       const int ct = cw * 32 + lane;
       float* aux = reinterpret_cast<float*>(smem + C::kAuxOff);
@@ -785,30 +860,38 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
           sq = __fdiv_rn(amax, 127.0f);
           const float rcp = amax != 0.0f ? __frcp_rn(sq) : 0.0f;
           for (int rr = ct; rr < kBM; rr += 64)
-            quant_row<D>(sQ(t), sQ8(t), i8_swz, rr, sq, rcp, amax == 0.0f);
+            quant_row<D>(sQ(t), sQ8(t), i8_swz, rr, sq, rcp);
           fence_proxy_async_smem();
         }
         if (ct == 0) sq_s[t] = sq;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[C::kBarQConv + t]);
       }
+      // K rows of this CTA's KV head: row j of the sequence at kg + j * kstr
+      const __half* kg = reinterpret_cast<const __half*>(p.k) +
+                         (static_cast<size_t>(start) * p.hkv + hk) * D;
+      const size_t kstr = static_cast<size_t>(p.hkv) * D;
+      uint8_t* k8ring = smem + C::kK8Ring0;
       for (int n = 0; n <= n_end && ok; ++n) {
-        const int ks = n % C::kKStages;
-        const bool got_k = mbar_wait(&bars[C::kBarK + ks],
-                                     (n / C::kKStages) & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, got_k)) {
-          ok = false;
-          break;
+        const int rs = n & 1;
+        // ring slot rs is free once both query tiles' Q K^T of tile n - 2
+        // completed
+        if (n >= 2) {
+          const bool got = mbar_wait(&bars[C::kBarK8Empty + rs],
+                                     ((n >> 1) - 1) & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, got)) {
+            ok = false;
+            break;
+          }
         }
-        uint32_t kinds = 0;
-        for (int t = 0; t < kQT; ++t)
-          kinds |= kinds_of(t, n, 0) | kinds_of(t, n, 1);
+        const uint32_t code = qk_code(0, n) | (qk_code(1, n) << 4);
         float sk = 0.0f;
-        if (kinds & kKindI8) {
-          uint8_t* kp = kslot(ks);
+        if (code & 0xccu) {
           float local = 0.0f;
           for (int rr = ct; rr < kBN; rr += 64)
-            if (n * kBN + rr < len) local = fmaxf(local, row_absmax_f16<D>(kp, rr));
+            if (n * kBN + rr < len)
+              local = fmaxf(local,
+                            row_absmax_global<D>(kg + (n * kBN + rr) * kstr));
           bool good = true;
           const float amax = block_max(local, good);
           if (!good) {
@@ -817,15 +900,17 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
           }
           sk = __fdiv_rn(amax, 127.0f);
           const float rcp = amax != 0.0f ? __frcp_rn(sk) : 0.0f;
+          uint8_t* k8 = k8ring + rs * C::kK8Bytes;
           for (int rr = ct; rr < kBN; rr += 64)
-            quant_row<D>(kp, kp + C::kK8Off, i8_swz, rr, sk, rcp,
-                         amax == 0.0f);
+            quant_row_global<D>(
+                n * kBN + rr < len ? kg + (n * kBN + rr) * kstr : nullptr, k8,
+                i8_swz, rr, sk, rcp);
           fence_proxy_async_smem();
         }
         if (ct == 0) sk_ring[n % C::kSkRing] = sk;
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&bars[C::kBarKConv + ks]);
+          mbar_arrive(&bars[C::kBarK8Full + rs]);
           mbar_arrive(&bars[C::kBarSK + n % C::kSkRing]);
         }
       }
@@ -986,7 +1071,9 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
         }
         // Lazy rescaling: keep the old max unless the tile exceeds it by
         // more than 2^threshold, so P <= 2^threshold stays in fp16 range.
-        const bool need = m_tile > m_run + kRescaleThreshold;
+        // (the fp16-accumulator study keeps P <= 1: fp16 O has no headroom)
+        const bool need =
+            m_tile > m_run + (p.pv_f16_acc ? 0.0f : kRescaleThreshold);
         const float m_old = m_run;
         if (need) {
           l_run *= ex2_approx(m_run - m_tile);
@@ -1027,9 +1114,17 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
             uint32_t o[32];
             tmem_ld32(lane_addr + C::kOCol + o0 + oc, o);
             tmem_ld_wait();
+            if (p.pv_f16_acc) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+              for (int j = 0; j < 32; ++j)
+                o[j] = __half_as_ushort(__float2half_rn(
+                    __half2float(__ushort_as_half(static_cast<uint16_t>(o[j]))) *
+                    alpha));
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            }
             tmem_st32(lane_addr + C::kOCol + o0 + oc, o);
           }
         }
@@ -1069,6 +1164,12 @@ __global__ void __launch_bounds__(threads_of(MODE), 1)
               uint32_t o[32];
               tmem_ld32(lane_addr + C::kOCol + o0 + oc, o);
               tmem_ld_wait();
+              if (p.pv_f16_acc) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  o[j] = __float_as_uint(__half2float(
+                      __ushort_as_half(static_cast<uint16_t>(o[j]))));
+              }
               uint32_t hv[16];
 #pragma unroll
               for (int j = 0; j < 16; ++j)

@@ -24,6 +24,13 @@ cudaError_t launch_quantize_blockwise(const void* x, const int32_t* cu_seqlens,
                                       float* scale, int32_t* status,
                                       cudaStream_t stream);
 
+// Q and K in one launch (the same results as one launch each).
+cudaError_t launch_quantize_blockwise_qk(
+    const void* q, const void* k, const int32_t* cu_seqlens, int batch,
+    int max_seqlen, int total_tokens, int hq, int hkv, int head_dim,
+    int block_q, int block_k, int8_t* q8, float* q_scale, int8_t* k8,
+    float* k_scale, int32_t* status, cudaStream_t stream);
+
 cudaError_t launch_pack_mask(const uint8_t* route, const int32_t* cu_seqlens,
                              int batch, int max_seqlen, int hkv, int block_m,
                              int block_n, int group, uint64_t* mask,
@@ -65,8 +72,7 @@ struct AttnParams {
   CUtensorMap tm_v;   // fp16 V  [T, hkv, d], box {64, 128, 1}
   CUtensorMap tm_v8;  // int8 V8 [T, hkv, d], box {d, 128, 1}, no swizzle
   CUtensorMap tm_o;   // fp16 O  [T, hq, d], box {64, 128, 1}, 128B swizzle
-  CUtensorMap tm_kh;  // fp16 K  [T, hkv, d], box {64, 64, 1}, 128B swizzle
-  CUtensorMap tm_kh8; // int8 K8 [T, hkv, d], box {d, 64, 1}
+  const uint16_t* k;  // fp16 K bits [T, hkv, d] (on-chip quantisation reads it)
   const int32_t* cu_seqlens;
   const int32_t* head_map;
   const uint64_t* mask;
@@ -87,7 +93,8 @@ struct AttnParams {
   int tiles_per_bit; // 64-key blocks per routing bit = g * route_bn / 64
   int quant_block_q, quant_block_k, nbq, nbk;
   int fp16_only;
-  int test_expire_wait;  // withhold the first V tile (timeout-path test)
+  int test_expire_wait;
+  int pv_f16_acc;  // study: O accumulated in fp16 (low half of each column)  // withhold the first V tile (timeout-path test)
   float scale_log2;  // softmax scale * log2(e)
 };
 

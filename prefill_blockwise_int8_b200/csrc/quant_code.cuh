@@ -63,6 +63,14 @@ __device__ __forceinline__ void quant_codes8(const float (&x)[8], float s,
   }
 }
 
+// Low bytes of four words (the code patterns above) -> one word, byte i
+// from word i.
+__device__ __forceinline__ uint32_t pack_low_bytes4(uint32_t a, uint32_t b,
+                                                    uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040),
+                     0x5410);
+}
+
 // The two fp16 halves of a 32-bit word as floats (exact).
 __device__ __forceinline__ void half2_bits_to_float2(uint32_t w, float& lo,
                                                      float& hi) {

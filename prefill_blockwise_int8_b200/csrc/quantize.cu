@@ -7,9 +7,12 @@
 // Per (sequence, head, block of tokens): scale = absmax / 127 (IEEE fp32
 // division), code = clamp(round_half_even(x / scale), -127, 127).
 //
-// HBM-bound: one CTA reads one block (up to 32 KB of fp16) once into
-// registers with 16-byte loads, reduces the absmax, and writes the codes
-// with 8-byte stores.  Rows of a block are strided by heads * d in memory,
+// HBM-bound: one CTA copies one block (up to 64 KB of fp16) once into
+// shared memory with 16-byte asynchronous copies (cp.async: few registers,
+// so six CTAs per SM keep their loads in flight together), reduces the
+// absmax, and writes the codes with 8-byte stores.  One launch can serve two tensors (Q and K): grid.y
+// runs over the heads of the first, then of the second, so both share one
+// grid and the short tail of a single launch is paid once.  Rows of a block are strided by heads * d in memory,
 // each row contiguous.  The per-element IEEE division is replaced by a
 // multiply with the reciprocal wherever that provably gives the same code,
 // and the integer code is read off a float's bit pattern (no conversion
@@ -25,20 +28,48 @@ namespace {
 
 constexpr int kQThreads = 256;
 
+// 16-byte global -> shared copy that bypasses L1 and registers; completes
+// for the issuing thread at cp_async_wait_all().
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+}
+
+// One tensor of a launch: x [T, heads, d] -> x8, scale [heads, batch, nblk].
+struct QuantJob {
+  const __half* x;
+  int8_t* x8;
+  float* scale;
+  int heads, block, nblk;
+};
+
 // VPT 16-byte vectors (8 halves) per thread; VPR vectors per row (d / 8),
-// 0 = taken from vpr_rt at run time.
+// 0 = taken from vpr_rt at run time.  Heads [0, j0.heads) of grid.y are
+// j0's, the rest j1's (j1.heads = 0 for a single tensor).
 template <int VPT, int VPR>
 __global__ void __launch_bounds__(kQThreads)
-    quantize_kernel(const __half* __restrict__ x,
+    quantize_kernel(const QuantJob j0, const QuantJob j1,
                     const int32_t* __restrict__ cu_seqlens, int batch,
-                    int max_seqlen, int total_tokens, int heads, int block,
-                    int nblk, int vpr_rt, int8_t* __restrict__ x8,
-                    float* __restrict__ scale, int32_t* status) {
+                    int max_seqlen, int total_tokens, int vpr_rt,
+                    int32_t* status) {
   const int vpr = VPR > 0 ? VPR : vpr_rt;
   const int d = vpr * 8;
+  const bool second = static_cast<int>(blockIdx.y) >= j0.heads;
+  const __half* __restrict__ x = second ? j1.x : j0.x;
+  int8_t* __restrict__ x8 = second ? j1.x8 : j0.x8;
+  float* __restrict__ scale = second ? j1.scale : j0.scale;
+  const int heads = second ? j1.heads : j0.heads;
+  const int block = second ? j1.block : j0.block;
+  const int nblk = second ? j1.nblk : j0.nblk;
   const int t = blockIdx.x;
-  const int h = blockIdx.y;
+  const int h = second ? blockIdx.y - j0.heads : blockIdx.y;
   const int b = blockIdx.z;
+  if (t >= nblk) return;
   const int start = cu_seqlens[b];
   const int len = cu_seqlens[b + 1] - start;
   if (start < 0 || len < 0 || len > max_seqlen || start + len > total_tokens) {
@@ -57,17 +88,27 @@ __global__ void __launch_bounds__(kQThreads)
   const __half* base = x + (static_cast<size_t>(start + r0) * heads + h) * d;
 
   // Consecutive threads take consecutive 16-byte vectors of a row, so each
-  // row's VPR vectors are one coalesced read.
-  uint4 v[VPT];
-  __half2 amax2 = __float2half2_rn(0.0f);
+  // row's VPR vectors are one coalesced read.  A thread only reads back the
+  // vectors it copied itself, so its own wait orders them.
+  extern __shared__ uint4 stage[];
 #pragma unroll
   for (int k = 0; k < VPT; ++k) {
     const int idx = threadIdx.x + k * kQThreads;
     if (idx < nv) {
       const int r = idx / vpr;
       const int c = idx % vpr;
-      v[k] = __ldg(reinterpret_cast<const uint4*>(base + r * row_stride) + c);
-      const __half2* hv = reinterpret_cast<const __half2*>(&v[k]);
+      cp_async16(&stage[idx],
+                 reinterpret_cast<const uint4*>(base + r * row_stride) + c);
+    }
+  }
+  cp_async_wait_all();
+  __half2 amax2 = __float2half2_rn(0.0f);
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const int idx = threadIdx.x + k * kQThreads;
+    if (idx < nv) {
+      const uint4 vk = stage[idx];
+      const __half2* hv = reinterpret_cast<const __half2*>(&vk);
 #pragma unroll
       for (int e = 0; e < 4; ++e) amax2 = __hmax2(amax2, __habs2(hv[e]));
     }
@@ -93,42 +134,58 @@ __global__ void __launch_bounds__(kQThreads)
     if (idx < nv) {
       const int r = idx / vpr;
       const int c = idx % vpr;
-      const uint32_t w4[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+      const uint4 vk = stage[idx];
+      const uint32_t w4[4] = {vk.x, vk.y, vk.z, vk.w};
       float f[8];
 #pragma unroll
       for (int e = 0; e < 4; ++e) half2_bits_to_float2(w4[e], f[2 * e], f[2 * e + 1]);
       uint32_t cb[8];
       quant_codes8(f, s, rcp, cb);
-      // low bytes of four patterns -> one word
-      auto pack4 = [](uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-        return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040),
-                           0x5410);
-      };
       *reinterpret_cast<uint2*>(qbase + r * row_stride + c * 8) =
-          make_uint2(pack4(cb[0], cb[1], cb[2], cb[3]),
-                     pack4(cb[4], cb[5], cb[6], cb[7]));
+          make_uint2(pack_low_bytes4(cb[0], cb[1], cb[2], cb[3]),
+                     pack_low_bytes4(cb[4], cb[5], cb[6], cb[7]));
     }
   }
 }
 
 template <int VPR>
 cudaError_t launch_vpr(dim3 grid, int vecs, cudaStream_t stream,
-                       const __half* x, const int32_t* cu_seqlens, int batch,
-                       int max_seqlen, int total_tokens, int heads, int block,
-                       int nblk, int vpr_rt, int8_t* x8, float* scale,
-                       int32_t* status) {
+                       const QuantJob& j0, const QuantJob& j1,
+                       const int32_t* cu_seqlens, int batch, int max_seqlen,
+                       int total_tokens, int vpr_rt, int32_t* status) {
   const int vpt = (vecs + kQThreads - 1) / kQThreads;
-#define TILEMIX_QLAUNCH(N)                                                  \
-  quantize_kernel<N, VPR><<<grid, kQThreads, 0, stream>>>(                  \
-      x, cu_seqlens, batch, max_seqlen, total_tokens, heads, block, nblk,   \
-      vpr_rt, x8, scale, status)
-  if (vpt <= 2) TILEMIX_QLAUNCH(2);
-  else if (vpt <= 4) TILEMIX_QLAUNCH(4);
-  else if (vpt <= 8) TILEMIX_QLAUNCH(8);
-  else if (vpt <= 16) TILEMIX_QLAUNCH(16);
-  else return cudaErrorInvalidValue;
-#undef TILEMIX_QLAUNCH
-  return cudaGetLastError();
+  const int smem = vecs * 16;  // one block of fp16, <= 64 KB
+  auto go = [&](auto kern) {
+    cudaError_t e = cudaFuncSetAttribute(
+        kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kQThreads, smem, stream>>>(j0, j1, cu_seqlens, batch,
+                                            max_seqlen, total_tokens, vpr_rt,
+                                            status);
+    return cudaGetLastError();
+  };
+  if (vpt <= 2) return go(quantize_kernel<2, VPR>);
+  if (vpt <= 4) return go(quantize_kernel<4, VPR>);
+  if (vpt <= 8) return go(quantize_kernel<8, VPR>);
+  if (vpt <= 16) return go(quantize_kernel<16, VPR>);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_jobs(const QuantJob& j0, const QuantJob& j1,
+                        const int32_t* cu_seqlens, int batch, int max_seqlen,
+                        int total_tokens, int head_dim, int32_t* status,
+                        cudaStream_t stream) {
+  dim3 grid(max(j0.nblk, j1.nblk), j0.heads + j1.heads, batch);
+  const int vecs = max(j0.block, j1.block) * head_dim / 8;
+  const int vpr = head_dim / 8;
+  if (head_dim == 128)
+    return launch_vpr<16>(grid, vecs, stream, j0, j1, cu_seqlens, batch,
+                          max_seqlen, total_tokens, vpr, status);
+  if (head_dim == 64)
+    return launch_vpr<8>(grid, vecs, stream, j0, j1, cu_seqlens, batch,
+                         max_seqlen, total_tokens, vpr, status);
+  return launch_vpr<0>(grid, vecs, stream, j0, j1, cu_seqlens, batch,
+                       max_seqlen, total_tokens, vpr, status);
 }
 
 }  // namespace
@@ -139,22 +196,24 @@ cudaError_t launch_quantize_blockwise(const void* x, const int32_t* cu_seqlens,
                                       int head_dim, int block, int8_t* x8,
                                       float* scale, int32_t* status,
                                       cudaStream_t stream) {
-  const int nblk = (max_seqlen + block - 1) / block;
-  dim3 grid(nblk, heads, batch);
-  const __half* xh = static_cast<const __half*>(x);
-  const int vecs = block * head_dim / 8;
-  const int vpr = head_dim / 8;
-  if (head_dim == 128)
-    return launch_vpr<16>(grid, vecs, stream, xh, cu_seqlens, batch,
-                          max_seqlen, total_tokens, heads, block, nblk, vpr,
-                          x8, scale, status);
-  if (head_dim == 64)
-    return launch_vpr<8>(grid, vecs, stream, xh, cu_seqlens, batch,
-                         max_seqlen, total_tokens, heads, block, nblk, vpr, x8,
-                         scale, status);
-  return launch_vpr<0>(grid, vecs, stream, xh, cu_seqlens, batch, max_seqlen,
-                       total_tokens, heads, block, nblk, vpr, x8, scale,
-                       status);
+  const QuantJob j0{static_cast<const __half*>(x), x8, scale, heads, block,
+                    (max_seqlen + block - 1) / block};
+  const QuantJob j1{nullptr, nullptr, nullptr, 0, 1, 0};
+  return launch_jobs(j0, j1, cu_seqlens, batch, max_seqlen, total_tokens,
+                     head_dim, status, stream);
+}
+
+cudaError_t launch_quantize_blockwise_qk(
+    const void* q, const void* k, const int32_t* cu_seqlens, int batch,
+    int max_seqlen, int total_tokens, int hq, int hkv, int head_dim,
+    int block_q, int block_k, int8_t* q8, float* q_scale, int8_t* k8,
+    float* k_scale, int32_t* status, cudaStream_t stream) {
+  const QuantJob jq{static_cast<const __half*>(q), q8, q_scale, hq, block_q,
+                    (max_seqlen + block_q - 1) / block_q};
+  const QuantJob jk{static_cast<const __half*>(k), k8, k_scale, hkv, block_k,
+                    (max_seqlen + block_k - 1) / block_k};
+  return launch_jobs(jq, jk, cu_seqlens, batch, max_seqlen, total_tokens,
+                     head_dim, status, stream);
 }
 
 }  // namespace tilemix

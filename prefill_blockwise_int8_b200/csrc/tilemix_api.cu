@@ -147,6 +147,43 @@ tilemix_status tilemix_quantize_blockwise(const void* x,
   return ok();
 }
 
+tilemix_status tilemix_quantize_blockwise_qk(
+    const void* q, const void* k, const int32_t* cu_seqlens, int batch,
+    int max_seqlen, int total_tokens, int hq, int hkv, int head_dim,
+    int block_q, int block_k, int8_t* q8, float* q_scale, int8_t* k8,
+    float* k_scale, int32_t* status, tilemix_stream_t stream) {
+  if (!q || !k || !cu_seqlens || !q8 || !q_scale || !k8 || !k_scale)
+    return fail(TILEMIX_ERR_INVALID_ARG, "quantize_qk: null pointer");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(q8, 16) ||
+      !aligned(k8, 16) || !aligned(q_scale, 4) || !aligned(k_scale, 4) ||
+      !aligned(cu_seqlens, 4) || (status && !aligned(status, 4)))
+    return fail(TILEMIX_ERR_INVALID_ARG, "quantize_qk: misaligned pointer");
+  if (batch < 0 || max_seqlen < 0 || total_tokens < 0 || hq <= 0 || hkv <= 0)
+    return fail(TILEMIX_ERR_INVALID_ARG, "quantize_qk: negative size");
+  if (head_dim <= 0 || head_dim % 8 != 0 || head_dim > 256)
+    return fail(TILEMIX_ERR_INVALID_ARG,
+                "quantize_qk: head_dim %d must be a multiple of 8 in [8, 256]",
+                head_dim);
+  for (int blk : {block_q, block_k})
+    if (blk <= 0 || blk > 256 || blk * head_dim > 32768)
+      return fail(TILEMIX_ERR_INVALID_ARG,
+                  "quantize_qk: block %d out of range (block*head_dim <= 32768)",
+                  blk);
+  if (batch == 0 || max_seqlen == 0) return ok();
+  if (static_cast<long long>(hq) + hkv > 65535 || batch > 65535)
+    return fail(TILEMIX_ERR_UNSUPPORTED,
+                "quantize_qk: hq + hkv or batch > 65535");
+  tilemix_status d = check_device();
+  if (d != TILEMIX_OK) return d;
+  cudaError_t e = tilemix::launch_quantize_blockwise_qk(
+      q, k, cu_seqlens, batch, max_seqlen, total_tokens, hq, hkv, head_dim,
+      block_q, block_k, q8, q_scale, k8, k_scale, status, stream);
+  if (e != cudaSuccess)
+    return fail(TILEMIX_ERR_CUDA, "quantize_qk launch: %s",
+                cudaGetErrorString(e));
+  return ok();
+}
+
 tilemix_status tilemix_pack_mask(const uint8_t* route,
                                  const int32_t* cu_seqlens, int batch,
                                  int max_seqlen, int hkv, int block_m,
@@ -358,7 +395,7 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   // With every tile FP16 there is nothing to quantise on chip.
   const bool on_chip = !fp16_only && (a->flags & TILEMIX_FLAG_QUANT_ON_CHIP) != 0;
   if (a->flags & ~(TILEMIX_FLAG_FP16_ONLY | TILEMIX_FLAG_QUANT_ON_CHIP |
-                   TILEMIX_FLAG_TEST_EXPIRE_WAIT))
+                   TILEMIX_FLAG_TEST_EXPIRE_WAIT | TILEMIX_FLAG_PV_F16_ACC))
     return fail(TILEMIX_ERR_INVALID_ARG, "attn: unknown flag bits 0x%x",
                 a->flags);
   if (a->kv_format != TILEMIX_KV_FP16 && a->kv_format != TILEMIX_KV_INT8)
@@ -457,8 +494,6 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   if (maps && !kv8)
     maps = make_map(&p.tm_k, a->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
                     a->hkv, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
-           make_map(&p.tm_kh, a->k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
-                    a->hkv, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
            make_map(&p.tm_v, a->v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, d, T,
                     a->hkv, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (maps && !fp16_only && !on_chip)
@@ -468,14 +503,13 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   // chip for FP16 groups) and V8 (converted to fp16 on chip).
   if (maps && (kv8 || (!fp16_only && !on_chip)))
     maps = make_map(&p.tm_k8, a->k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
-                    a->hkv, d, 128, i8sw) &&
-           make_map(&p.tm_kh8, a->k8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
-                    a->hkv, d, 64, i8sw);
+                    a->hkv, d, 128, i8sw);
   if (maps && kv8)
     maps = make_map(&p.tm_v8, a->v8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, T,
                     a->hkv, d, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!maps) return fail(TILEMIX_ERR_CUDA, "attn: tensor map encoding failed");
 
+  p.k = kv8 ? nullptr : static_cast<const uint16_t*>(a->k);
   p.cu_seqlens = a->cu_seqlens;
   p.head_map = a->head_map;
   p.mask = fp16_only ? nullptr : a->mask;
@@ -504,6 +538,7 @@ tilemix_status tilemix_attn_prefill(const tilemix_attn_params* a,
   p.nbk = (a->max_seqlen + qbk - 1) / qbk;
   p.fp16_only = fp16_only ? 1 : 0;
   p.test_expire_wait = (a->flags & TILEMIX_FLAG_TEST_EXPIRE_WAIT) ? 1 : 0;
+  p.pv_f16_acc = (a->flags & TILEMIX_FLAG_PV_F16_ACC) ? 1 : 0;
   const float scale =
       a->softmax_scale > 0.0f ? a->softmax_scale : 1.0f / std::sqrt(float(d));
   p.scale_log2 = scale * 1.4426950408889634f;

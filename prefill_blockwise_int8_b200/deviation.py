@@ -14,8 +14,12 @@ draw exactly round(c * N_legal) INT8 groups per KV head.
     python -m prefill_blockwise_int8_b200.deviation --policies band,adaptive
 
 With --policies it compares routing policies (the static templates and the
-adaptive one) at equal per-row INT8 shares instead.  Needs a GPU; prints
-one line per coverage (and policy) and returns the rows.
+adaptive one) at equal per-row INT8 shares instead.  The accumulation axis
+(appendix G.4 of the same summary: FP16 against FP32 accumulation) repeats
+each coverage with O accumulated in fp16 (the study-only
+TILEMIX_FLAG_PV_F16_ACC), still measured against the fp32-accumulated
+all-FP16 reference.  Needs a GPU; prints one line per coverage (and policy
+or accumulator) and returns the rows.
 """
 from __future__ import annotations
 
@@ -31,9 +35,12 @@ DEFAULT_COVERAGES = (0.0, 0.05, 0.10, 0.25, 0.50, 0.75, 1.0)
 POLICIES = ("row_random", "band", "bigbird", "sptrans", "adaptive")
 
 
+ACCUMULATORS = ("f32", "f16")
+
+
 def run(seqlen: int = 8192, hq: int = 8, hkv: int = 2, d: int = 128,
         block_m: int = 128, block_n: int = 128, coverages=DEFAULT_COVERAGES,
-        seed: int = 7, device: str = "cuda"):
+        seed: int = 7, device: str = "cuda", accumulators=("f32",)):
     import torch
 
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -62,12 +69,15 @@ def run(seqlen: int = 8192, hq: int = 8, hkv: int = 2, d: int = 128,
         w = base.with_(coverage=float(c), mask_seed=seed + 1 + int(c * 1000))
         route = torch.from_numpy(W.route_bytes(w, inp["seqlens"])).to(dev)
         mask = tm.tilemix_pack_mask(route, cu, ms, block_m, block_n, g)
-        out = tm.tilemix_attn_prefill(
-            q, k, v, cu, ms, q8=q8, q_scale=sq, k8=k8, k_scale=sk, mask=mask,
-            block_m=block_m, block_n=block_n, group=g).float()
-        diff = (out - ref).abs()
-        rows.append(dict(coverage=float(c), max_diff=float(diff.max()),
-                         mean_diff=float(diff.mean())))
+        for acc in accumulators:
+            out = tm.tilemix_attn_prefill(
+                q, k, v, cu, ms, q8=q8, q_scale=sq, k8=k8, k_scale=sk,
+                mask=mask, block_m=block_m, block_n=block_n, group=g,
+                pv_f16_acc=(acc == "f16")).float()
+            diff = (out - ref).abs()
+            rows.append(dict(coverage=float(c), accumulate=acc,
+                             max_diff=float(diff.max()),
+                             mean_diff=float(diff.mean())))
     return rows
 
 
@@ -135,6 +145,9 @@ def main(argv=None):
                     help="comma list of " + ",".join(POLICIES) + ": compare "
                          "routing policies at per-row INT8 shares instead of "
                          "the per-KV-head random masks")
+    ap.add_argument("--accumulate", default="f32",
+                    help="comma list of " + ",".join(ACCUMULATORS) + ": the "
+                         "P V accumulator(s) to measure (f16 is study only)")
     args = ap.parse_args(argv)
     if args.policies:
         pols = tuple(p for p in args.policies.split(",") if p)
@@ -146,12 +159,17 @@ def main(argv=None):
             print(f"{r['coverage']:>14.2f} {r['policy']:>11} "
                   f"{r['max_diff']:>10.3e} {r['mean_diff']:>10.3e}")
         return rows
+    accs = tuple(a for a in args.accumulate.split(",") if a)
+    bad = [a for a in accs if a not in ACCUMULATORS]
+    if bad:
+        raise SystemExit(f"unknown accumulator(s) {bad}")
     rows = run(seqlen=args.seqlen, hq=args.hq, hkv=args.hkv,
-               block_n=args.block_n)
-    print(f"{'INT8 coverage':>14} {'MaxDiff':>10} {'MeanDiff':>10}")
+               block_n=args.block_n, accumulators=accs)
+    print(f"{'INT8 coverage':>14} {'P V acc':>8} {'MaxDiff':>10} "
+          f"{'MeanDiff':>10}")
     for r in rows:
-        print(f"{r['coverage']:>14.2f} {r['max_diff']:>10.3e} "
-              f"{r['mean_diff']:>10.3e}")
+        print(f"{r['coverage']:>14.2f} {r['accumulate']:>8} "
+              f"{r['max_diff']:>10.3e} {r['mean_diff']:>10.3e}")
     return rows
 
 

@@ -67,6 +67,48 @@ def test_quantize_bitexact_varlen(tm, d, block):
     assert np.array_equal(gs.cpu().numpy().view(np.uint32), refs.view(np.uint32))
 
 
+@pytest.mark.parametrize("qb,kb", [(128, 128), (64, 128), (128, 32)])
+def test_quantize_qk_one_launch_bitexact(tm, qb, kb):
+    """Q and K in one launch: byte-exact to the oracle for each tensor (and
+    so to two single launches), with different heads and block sizes."""
+    lens = np.array([1, 127, 128, 129, 300, 0, 1000], dtype=np.int32)
+    cu = W.cu_seqlens(lens)
+    rng = np.random.default_rng(qb + 3 * kb)
+    q = (rng.standard_normal((lens.sum(), 6, 128)) * 4).astype(np.float16)
+    k = (rng.standard_normal((lens.sum(), 2, 128)) * 4).astype(np.float16)
+    k[cu[4]:cu[4] + 2, 1, 3] = -500.0  # an outlier
+    q[cu[2]:cu[3], 4, :] = 0           # an all-zero block
+    ms = int(lens.max())
+    rq8, rqs = oracle.quantize_blockwise(q, cu, ms, qb)
+    rk8, rks = oracle.quantize_blockwise(k, cu, ms, kb)
+    q8, qs, k8, ks = tm.tilemix_quantize_blockwise_qk(
+        dev_tensor(q), dev_tensor(k), dev_tensor(cu), ms, qb, kb)
+    torch.cuda.synchronize()
+    assert np.array_equal(q8.cpu().numpy(), rq8)
+    assert np.array_equal(k8.cpu().numpy(), rk8)
+    assert np.array_equal(qs.cpu().numpy().view(np.uint32), rqs.view(np.uint32))
+    assert np.array_equal(ks.cpu().numpy().view(np.uint32), rks.view(np.uint32))
+
+
+def test_quantize_qk_full_size_equals_single_launches(tm):
+    """At the LLaMA-3.2-3B prefill shape the one-launch codes and scales
+    equal those of one launch per tensor (which the test above and the
+    single-tensor tests pin to the oracle)."""
+    w = W.LLAMA32_3B_4K
+    inp = W.make(w)
+    cu = dev_tensor(inp["cu_seqlens"])
+    q, k = dev_tensor(inp["q"]), dev_tensor(inp["k"])
+    ms = inp["max_seqlen"]
+    q8a, qsa = tm.tilemix_quantize_blockwise(q, cu, ms, w.quant_block_q)
+    k8a, ksa = tm.tilemix_quantize_blockwise(k, cu, ms, w.quant_block_k)
+    q8b, qsb, k8b, ksb = tm.tilemix_quantize_blockwise_qk(
+        q, k, cu, ms, w.quant_block_q, w.quant_block_k)
+    torch.cuda.synchronize()
+    assert torch.equal(q8a, q8b) and torch.equal(k8a, k8b)
+    assert torch.equal(qsa.view(torch.int32), qsb.view(torch.int32))
+    assert torch.equal(ksa.view(torch.int32), ksb.view(torch.int32))
+
+
 def test_quantize_golden_ties(tm):
     here = os.path.dirname(__file__)
     cases = json.load(open(os.path.join(here, "golden",
