@@ -90,16 +90,30 @@ struct ExactSums {
     run = 0;
   }
   // rows first, first + step, ... < last of a [rows, stride] fp16 matrix,
-  // 16-byte chunk at `base`
+  // 16-byte chunk at `base`.  Eight rows at a time: their loads are issued
+  // together, so each thread keeps 128 bytes in flight.
   __device__ __forceinline__ void add_rows(const uint16_t* __restrict__ base,
                                            size_t stride, int first, int last,
                                            int step) {
+    constexpr int kBatch = 8;  // kExactRun is a multiple of it
     const uint16_t* p = base + static_cast<size_t>(first) * stride;
     const size_t dp = static_cast<size_t>(step) * stride;
-#pragma unroll 4
-    for (int i = first; i < last; i += step, p += dp) {
+    int i = first;
+    for (; i + (kBatch - 1) * step < last; i += kBatch * step) {
+      uint4 w[kBatch];
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r)
+        w[r] = __ldg(reinterpret_cast<const uint4*>(p + r * dp));
+      p += kBatch * dp;
+      if (run + kBatch > kExactRun) settle();
+#pragma unroll
+      for (int r = 0; r < kBatch; ++r) add_chunk(a, w[r]);
+      run += kBatch;
+    }
+    for (; i < last; i += step, p += dp) {
+      if (run == kExactRun) settle();
       add_chunk(a, __ldg(reinterpret_cast<const uint4*>(p)));
-      if (++run == kExactRun) settle();
+      ++run;
     }
   }
 };
@@ -189,9 +203,11 @@ __global__ void __launch_bounds__(kSumThreads)
   }
 }
 
-// One CTA of 64 threads per (sequence, KV head, query-tile row); thread j
-// computes the statistic of group j over all channels in 24-bit limbs:
-// with Sq = a1 * 2^24 + a0 and Sk = b1 * 2^24 + b0 (0 <= a0, b0 < 2^24),
+// One CTA per (sequence, KV head, run of kRankRows query-tile rows): the
+// key groups' sums are staged once in shared memory as 24-bit limbs, then
+// four rows at a time, 64 threads each: thread j computes the statistic of
+// group j over all channels, with Sq = a1 * 2^24 + a0 and Sk = b1 * 2^24 +
+// b0 (0 <= a0, b0 < 2^24),
 //   Sq . Sk = 2^48 sum a1 b1 + 2^24 sum (a0 b1 + a1 b0) + sum a0 b0.
 // The host admits only tiles with rows, keys < 2^15, rows * d and keys * d
 // < 2^22 and rows * keys * d < 2^47 (rows = query rows of a tile times its
@@ -199,20 +215,35 @@ __global__ void __launch_bounds__(kSumThreads)
 // 2^40 keys: the limbs fit int32, the three low sums int64 (their sum
 // included), and the statistic int128.  Thread j then ranks group j, writes
 // its byte, and warp ballots give the routing word.
-__global__ void __launch_bounds__(64)
+constexpr int kRankRows = 8;
+constexpr int kRankLanes = 4;  // rows in flight, 64 threads each
+constexpr int kKPitch = kGroups + 1;  // int2 per channel row of the stage
+
+__host__ __device__ constexpr int rank_smem_bytes(int d) {
+  return d * kKPitch * static_cast<int>(sizeof(int2));
+}
+
+__device__ __forceinline__ int2 limbs24(int64_t v) {
+  return make_int2(static_cast<int>(v & 0xFFFFFF), static_cast<int>(v >> 24));
+}
+
+__global__ void __launch_bounds__(64 * kRankLanes)
     rank_kernel(const int32_t* __restrict__ cu_seqlens,
                 const int32_t* __restrict__ head_map, int hq, int max_seqlen,
                 int total_tokens, int hkv, int tm, int d, int block_m,
                 int block_n, int group, int permille,
                 const int64_t* __restrict__ sq, const int64_t* __restrict__ sk,
                 uint8_t* __restrict__ route, uint64_t* __restrict__ mask) {
-  __shared__ int2 q_s[256];  // (a0, a1) per channel
-  __shared__ __int128 imp_s[kGroups];
-  const int j = threadIdx.x;
-  const int lane = j & 31;
-  const long long row = blockIdx.x;  // (b * hkv + hk) * tm + m
-  const int m = static_cast<int>(row % tm);
-  const long long bh = row / tm;
+  extern __shared__ int2 k_s[];  // [channel][kKPitch]: group j at column j
+  __shared__ int2 q_s[kRankLanes][256];
+  __shared__ __int128 imp_s[kRankLanes][kGroups];
+  const int tid = threadIdx.x;
+  const int rl = tid >> 6;  // row lane
+  const int j = tid & 63;
+  const int lane = tid & 31;
+  const int chunks = (tm + kRankRows - 1) / kRankRows;
+  const long long bh = blockIdx.x / chunks;  // b * hkv + hk
+  const int m0 = static_cast<int>(blockIdx.x % chunks) * kRankRows;
   const int b = static_cast<int>(bh / hkv);
   const int start = cu_seqlens[b];
   const int len = cu_seqlens[b + 1] - start;
@@ -221,56 +252,60 @@ __global__ void __launch_bounds__(64)
   // is then written as 0, like the rows of an invalid sequence.
   bool bad_map = false;
   if (head_map)
-    for (int h = j; h < hq; h += 64) {
+    for (int h = tid; h < hq; h += blockDim.x) {
       const int hm = head_map[h];
       bad_map |= hm < 0 || hm >= hkv;
     }
   bad_map = __syncthreads_or(bad_map) != 0;
-  int G = 0;  // an invalid sequence was reported by the first pass
-  if (!bad_map && start >= 0 && len >= 0 && len <= max_seqlen &&
-      start + len <= total_tokens && static_cast<long long>(m) * block_m < len)
-    G = ((min((m + 1) * block_m, len) - 1) / block_n) / group + 1;
-  for (int c = j; c < d; c += 64) {
-    const int64_t v = sq[row * d + c];
-    q_s[c] = make_int2(static_cast<int>(v & 0xFFFFFF), static_cast<int>(v >> 24));
+  const bool seq_ok = !bad_map && start >= 0 && len >= 0 &&
+                      len <= max_seqlen && start + len <= total_tokens;
+  // key sums of the 64 groups, read along channels (coalesced)
+  const int64_t* skb = sk + bh * kGroups * d;
+  for (int i = tid; i < kGroups * d; i += blockDim.x) {
+    const int g = i / d, c = i - g * d;
+    k_s[c * kKPitch + g] = limbs24(skb[i]);
   }
-  __syncthreads();
-  if (j < G) {
-    const longlong2* kg =
-        reinterpret_cast<const longlong2*>(sk + (bh * kGroups + j) * d);
-    int64_t lo = 0, mid = 0;
-    __int128 hi = 0;
+  for (int it = 0; it < kRankRows / kRankLanes; ++it) {
+    const int m = m0 + it * kRankLanes + rl;
+    const bool row_ok = m < tm;
+    const long long row = bh * tm + m;
+    int G = 0;  // an invalid sequence was reported by the first pass
+    if (row_ok && seq_ok && static_cast<long long>(m) * block_m < len)
+      G = ((min((m + 1) * block_m, len) - 1) / block_n) / group + 1;
+    if (row_ok)
+      for (int c = j; c < d; c += 64) q_s[rl][c] = limbs24(sq[row * d + c]);
+    __syncthreads();
+    if (j < G) {
+      int64_t lo = 0, mid = 0;
+      __int128 hi = 0;
 #pragma unroll 4
-    for (int c2 = 0; c2 < (d >> 1); ++c2) {
-      const longlong2 kv = __ldg(kg + c2);
-      const int64_t kk[2] = {kv.x, kv.y};
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int2 a = q_s[2 * c2 + e];
-        const int b0 = static_cast<int>(kk[e] & 0xFFFFFF);
-        const int b1 = static_cast<int>(kk[e] >> 24);
-        lo += static_cast<int64_t>(a.x) * b0;
-        mid += static_cast<int64_t>(a.x) * b1 + static_cast<int64_t>(a.y) * b0;
-        hi += static_cast<int64_t>(a.y) * b1;
+      for (int c = 0; c < d; ++c) {
+        const int2 a = q_s[rl][c];
+        const int2 k = k_s[c * kKPitch + j];
+        lo += static_cast<int64_t>(a.x) * k.x;
+        mid += static_cast<int64_t>(a.x) * k.y + static_cast<int64_t>(a.y) * k.x;
+        hi += static_cast<int64_t>(a.y) * k.y;
       }
+      imp_s[rl][j] = (hi << 48) + (static_cast<__int128>(mid) << 24) + lo;
     }
-    imp_s[j] = (hi << 48) + (static_cast<__int128>(mid) << 24) + lo;
-  }
-  __syncthreads();
-  const int k_fp16 = G - (permille * G + 500) / 1000;
-  uint8_t bit = 0;
-  if (j < G) {
-    const __int128 v = imp_s[j];
-    int rank = 0;  // groups ahead of j: a larger statistic, or equal and smaller index
-    for (int i = 0; i < G; ++i) {
-      const __int128 x = imp_s[i];
-      rank += (x > v || (x == v && i < j)) ? 1 : 0;
+    __syncthreads();
+    const int k_fp16 = G - (permille * G + 500) / 1000;
+    uint8_t bit = 0;
+    if (j < G) {
+      const __int128 v = imp_s[rl][j];
+      int rank = 0;  // groups ahead of j: a larger statistic, or equal and smaller index
+      for (int i = 0; i < G; ++i) {
+        const __int128 x = imp_s[rl][i];
+        rank += (x > v || (x == v && i < j)) ? 1 : 0;
+      }
+      bit = rank >= k_fp16 ? 1 : 0;
     }
-    bit = rank >= k_fp16 ? 1 : 0;
+    if (row_ok && route) route[row * 64 + j] = bit;
+    const uint32_t half = __ballot_sync(0xffffffffu, bit != 0);
+    if (row_ok && mask && lane == 0)
+      reinterpret_cast<uint32_t*>(mask + row)[j >> 5] = half;
+    __syncthreads();  // q_s and imp_s are rewritten by the next rows
   }
-  if (route) route[row * 64 + j] = bit;
-  const uint32_t half = __ballot_sync(0xffffffffu, bit != 0);
-  if (mask && lane == 0) reinterpret_cast<uint32_t*>(mask + row)[j >> 5] = half;
 }
 
 }  // namespace
@@ -320,8 +355,13 @@ cudaError_t launch_route_adaptive(const void* q, const void* k,
       kpg, gpc, sq, sk, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const long long rows = static_cast<long long>(batch) * hkv * tm;
-  rank_kernel<<<static_cast<unsigned>(rows), 64, 0, stream>>>(
+  const long long ctas = static_cast<long long>(batch) * hkv *
+                         ((tm + kRankRows - 1) / kRankRows);
+  const int smem = rank_smem_bytes(d);
+  e = cudaFuncSetAttribute(rank_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  rank_kernel<<<static_cast<unsigned>(ctas), 64 * kRankLanes, smem, stream>>>(
       cu_seqlens, head_map, hq, max_seqlen, total_tokens, hkv, tm, d, block_m,
       block_n, group, permille, sq, sk, route, mask);
   return cudaGetLastError();
