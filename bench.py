@@ -53,7 +53,7 @@ INT8_OVER_FP16 = 2.0  # nominal dense INT8 / FP16 tensor ratio (4.5 / 2.25 P)
 # this bench's own command, keyed by workload and by a hash of the kernel
 # sources the capture ran; a changed kernel reports null until re-captured.
 NCU_TRAFFIC = {
-    ("llama32_3b_b8_L4096_int8_75", "5fe750a12f3edf50"): 466_603_520 + 177_182_208,
+    ("llama32_3b_b8_L4096_int8_75", "2625fb088d1686fc"): 466_481_920 + 178_798_080,
 }
 KERNEL_SOURCES = ("prefill_blockwise_int8_b200/csrc/attn_prefill.cu",
                   "prefill_blockwise_int8_b200/csrc/ptx.cuh",
@@ -63,8 +63,8 @@ KERNEL_SOURCES = ("prefill_blockwise_int8_b200/csrc/attn_prefill.cu",
 # the same for the two adaptive-routing kernels (sums + rank, per call)
 ROUTE_SOURCES = ("prefill_blockwise_int8_b200/csrc/route_adaptive.cu",)
 ROUTE_TRAFFIC = {
-    ("llama32_3b_b8_L4096_int8_75", "3191f6e23b13a14a"):
-        268_517_632 + 8_055_808 + 6_310_400,
+    ("llama32_3b_b8_L4096_int8_75", "5a599996a59ca2de"):
+        268_482_816 + 7_033_344 + 6_314_752,
 }
 
 
@@ -403,13 +403,17 @@ def run_gpu(args):
     set0 = dict(q=q, k=k, v=v, cu=cu, route=route, k8=k8, k_scale=sk, v8=v8,
                 v_scale=sv, out=out)
 
-    def step(attn_events=None, route_events=None, b=None):
+    def step(attn_events=None, route_events=None, b=None, quant_events=None):
         b = set0 if b is None else b
         if not kv8 and not on_chip:  # Q and K in one launch
+            if quant_events:
+                quant_events[0].record(stream)
             tm.tilemix_quantize_blockwise_qk(
                 b["q"], b["k"], b["cu"], ms, w.quant_block_q, w.quant_block_k,
                 q8=q8, q_scale=sq, k8=b["k8"], k_scale=b["k_scale"],
                 status=status)
+            if quant_events:
+                quant_events[1].record(stream)
         elif not on_chip:
             tm.tilemix_quantize_blockwise(b["q"], b["cu"], ms, w.quant_block_q,
                                           x8=q8, scale=sq, status=status)
@@ -443,7 +447,7 @@ def run_gpu(args):
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()} during warmup")
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)]
           for _ in range(args.steps)]
     smi_index = local
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
@@ -458,7 +462,8 @@ def run_gpu(args):
         for i in range(args.steps):
             flush.zero_()
             ev[i][0].record(stream)
-            step((ev[i][1], ev[i][2]), (ev[i][4], ev[i][5]))
+            step((ev[i][1], ev[i][2]), (ev[i][4], ev[i][5]),
+                 quant_events=(ev[i][6], ev[i][7]))
             ev[i][3].record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
@@ -466,6 +471,8 @@ def run_gpu(args):
     step_ms = [e[0].elapsed_time(e[3]) for e in ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
     route_ms = [e[4].elapsed_time(e[5]) for e in ev]
+    quant_ms = ([e[6].elapsed_time(e[7]) for e in ev]
+                if not kv8 and not on_chip else None)
     total_ms = max_over_ranks(sum(step_ms), dev)
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()} in timed region")
@@ -586,6 +593,21 @@ def run_gpu(args):
                       "traffic": measured_route_traffic(w.name),
                       "kernels": "sums_kernel + rank_kernel"}
 
+    quant_roof = None
+    if quant_ms:
+        # Q and K read once as fp16, Q8 and K8 written once, fp32 scales
+        nq = -(-ms // w.quant_block_q) * w.hq * len(lens)
+        nk = -(-ms // w.quant_block_k) * w.hkv * len(lens)
+        nbytes = T * (w.hq + w.hkv) * w.d * 3 + 4 * (nq + nk)
+        q_s = statistics.mean(quant_ms) * 1e-3
+        gbs = nbytes / q_s / 1e9
+        quant_roof = {"bound": "hbm", "achieved": round(gbs, 1),
+                      "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                      "frac": round(gbs / float(peaks["hbm_gbs"]), 4),
+                      "bytes_per_launch": nbytes,
+                      "ms": round(q_s * 1e3, 4),
+                      "kernel": "quantize_kernel (Q and K, one launch)"}
+
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         rate, desc, cores = oracle_sample_rate(inp, args.cpu_seconds)
@@ -602,6 +624,7 @@ def run_gpu(args):
                                   permille=permille),
         "routing_ms": round(statistics.mean(route_ms), 4),
         "routing_roofline": route_roof,
+        "quantiser_roofline": quant_roof,
         "effective_tflops": wk["effective"] / (ms_step * 1e-3) / 1e12 * world,
         "attn_effective_tflops": achieved,
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,

@@ -66,17 +66,19 @@ __device__ __forceinline__ void add_chunk(double (&a)[8], uint4 w) {
 }
 
 // Running exact sums of one thread's eight channels: doubles for runs of at
-// most kExactRun rows, then int64 totals of value * 2^24.
+// most kExactRun rows, then int64 totals of value * 2^24.  The totals live
+// in shared memory (t[e * kSumThreads], one column per thread): they change
+// once per run, and the registers they would take go to loads in flight.
 struct ExactSums {
   double a[8];
-  int64_t t[8];
+  int64_t* t;
   int run;
 
   __device__ __forceinline__ void clear() {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       a[e] = 0.0;
-      t[e] = 0;
+      t[e * kSumThreads] = 0;
     }
     run = 0;
   }
@@ -84,7 +86,7 @@ struct ExactSums {
     // 2^1032 in two exact power-of-two steps (2^1032 is not a double)
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      t[e] += __double2ll_rn(a[e] * 0x1p1000 * 0x1p32);
+      t[e * kSumThreads] += __double2ll_rn(a[e] * 0x1p1000 * 0x1p32);
       a[e] = 0.0;
     }
     run = 0;
@@ -125,7 +127,7 @@ __device__ __forceinline__ void reduce_slices(const ExactSums& s,
                                               int64_t* __restrict__ out) {
   if (rs < slices) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) part_s[rs * d + cc * 8 + e] = s.t[e];
+    for (int e = 0; e < 8; ++e) part_s[rs * d + cc * 8 + e] = s.t[e * kSumThreads];
   }
   __syncthreads();
   for (int c = threadIdx.x; c < d; c += kSumThreads) {
@@ -161,7 +163,9 @@ __global__ void __launch_bounds__(kSumThreads)
   if (!valid && threadIdx.x == 0 && u == 0 && hk == 0)
     report_status(status, kStatusBadSeqlens);
   const bool active = valid && rs < slices;
+  __shared__ int64_t totals_s[8 * kSumThreads];
   ExactSums s;
+  s.t = totals_s + threadIdx.x;
   s.clear();
   if (u < tm) {
     if (active) {
@@ -215,7 +219,7 @@ __global__ void __launch_bounds__(kSumThreads)
 // 2^40 keys: the limbs fit int32, the three low sums int64 (their sum
 // included), and the statistic int128.  Thread j then ranks group j, writes
 // its byte, and warp ballots give the routing word.
-constexpr int kRankRows = 8;
+constexpr int kRankRows = 4;
 constexpr int kRankLanes = 4;  // rows in flight, 64 threads each
 constexpr int kKPitch = kGroups + 1;  // int2 per channel row of the stage
 
@@ -259,11 +263,27 @@ __global__ void __launch_bounds__(64 * kRankLanes)
   bad_map = __syncthreads_or(bad_map) != 0;
   const bool seq_ok = !bad_map && start >= 0 && len >= 0 &&
                       len <= max_seqlen && start + len <= total_tokens;
-  // key sums of the 64 groups, read along channels (coalesced)
-  const int64_t* skb = sk + bh * kGroups * d;
-  for (int i = tid; i < kGroups * d; i += blockDim.x) {
-    const int g = i / d, c = i - g * d;
-    k_s[c * kKPitch + g] = limbs24(skb[i]);
+  // key sums of the 64 groups, read along channels (coalesced, 16 bytes
+  // per thread and eight loads in flight: 64 * d / 2 is a multiple of the
+  // block size for d a multiple of 8)
+  const longlong2* skb = reinterpret_cast<const longlong2*>(sk + bh * kGroups * d);
+  const int n2 = kGroups * d / 2;
+  for (int i0 = tid; i0 < n2; i0 += 8 * blockDim.x) {
+    longlong2 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      v[u] = i < n2 ? __ldg(skb + i) : make_longlong2(0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < n2) {
+        const int g = (2 * i) / d, c = 2 * i - g * d;
+        k_s[c * kKPitch + g] = limbs24(v[u].x);
+        k_s[(c + 1) * kKPitch + g] = limbs24(v[u].y);
+      }
+    }
   }
   for (int it = 0; it < kRankRows / kRankLanes; ++it) {
     const int m = m0 + it * kRankLanes + rl;
