@@ -163,6 +163,34 @@ def test_quantize_and_pack_host_checks():
     assert pk(None, FAKE, 1, 128, 1, 64, 64, 1, FAKE, None, None) == INVALID
 
 
+def test_quantize_qk_host_checks():
+    # (q, k, cu, batch, max_seqlen, T, hq, hkv, d, block_q, block_k,
+    #  q8, q_scale, k8, k_scale, status, stream)
+    qk = tm.lib.tilemix_quantize_blockwise_qk
+    good = [FAKE, FAKE, FAKE, 1, 128, 128, 6, 2, 128, 128, 128,
+            FAKE, FAKE, FAKE, FAKE, None, None]
+
+    def call(**over):
+        a = list(good)
+        names = ["q", "k", "cu", "batch", "ms", "T", "hq", "hkv", "d", "bq",
+                 "bk", "q8", "qs", "k8", "ks", "status", "stream"]
+        for nm, v in over.items():
+            a[names.index(nm)] = v
+        return qk(*a)
+
+    assert call(k=None) == INVALID
+    assert call(k8=None) == INVALID
+    assert call(q=FAKE + 8) == INVALID          # not 16-byte aligned
+    assert call(ks=FAKE + 2) == INVALID         # not 4-byte aligned
+    assert call(hkv=0) == INVALID
+    assert call(d=60) == INVALID
+    assert call(bk=300) == INVALID
+    assert call(d=256, bq=256) == INVALID       # block * d > 32768
+    assert call(hq=65535, hkv=1) == UNSUPPORTED
+    assert call(batch=0, ms=0) == OK            # nothing to do, nothing launched
+    assert accepted(qk, *good)
+
+
 def test_route_template_host_checks():
     rt = tm.lib.tilemix_route_template
     # layout, int8_permille, seed, cu, batch, max_seqlen, hkv, bm, bn, g, route
@@ -231,6 +259,7 @@ def test_binding_refuses_host_tensors_no_cpu_fallback():
     route = torch.zeros((1, 1, 1, 64), dtype=torch.uint8)
     calls = [
         lambda: tm.tilemix_quantize_blockwise(x, cu, 4, 128),
+        lambda: tm.tilemix_quantize_blockwise_qk(x, k, cu, 4, 128, 128),
         lambda: tm.tilemix_pack_mask(route, cu, 4, 64, 64, 1),
         lambda: tm.tilemix_route_template("band", 500, cu, 4, 1, 64, 64, 1),
         lambda: tm.tilemix_route_adaptive(x, k, cu, 4, 64, 64, 1, 500),
