@@ -127,6 +127,7 @@ def test_attn_host_checks_accept_a_valid_call():
     ("mask", 0, INVALID),             # routed mode needs the words
     ("quant_block_k", 96, UNSUPPORTED),     # not a multiple of block_n
     ("flags", 0x80, INVALID),
+    ("flags", 0x10, INVALID),         # the first undefined bit
 ])
 def test_attn_host_checks_reject(field, value, expect):
     assert call(good_params(**{field: value})) == expect
@@ -140,6 +141,24 @@ def test_attn_block_m64_needs_block_n64():
 def test_attn_fp16_only_needs_no_int8_operands():
     p = good_params(flags=tm.FLAG_FP16_ONLY, mask=0, q8=0, k8=0, q_scale=0,
                     k_scale=0)
+    assert accepted(call, p)
+
+
+def test_flag_values_match_the_header():
+    text = open(os.path.join(ROOT, "include", "tilemix.h")).read()
+    flags = dict(re.findall(r"#define TILEMIX_FLAG_(\w+) (\d+)u", text))
+    assert flags, "no TILEMIX_FLAG_ defines found"
+    for name, value in flags.items():
+        assert getattr(tm, "FLAG_" + name) == int(value), name
+
+
+def test_attn_study_flag_is_accepted():
+    # TILEMIX_FLAG_PV_F16_ACC (study only) passes the host checks, alone
+    # and with the FP16-only reference mode
+    assert tm.FLAG_PV_F16_ACC == 8
+    assert accepted(call, good_params(flags=tm.FLAG_PV_F16_ACC))
+    p = good_params(flags=tm.FLAG_PV_F16_ACC | tm.FLAG_FP16_ONLY, mask=0,
+                    q8=0, k8=0, q_scale=0, k_scale=0)
     assert accepted(call, p)
 
 
